@@ -1,0 +1,173 @@
+"""B200 (sm_100a) attention for Stable Diffusion's UNet transformer blocks.
+
+    O = softmax(scale * Q K^T) V,   Q [B,H,N,d], K and V [B,H,M,d], d in {40, 80, 160}
+
+Two forms, after "Speed Is All You Need: On-Device Acceleration of Large
+Diffusion Models via GPU-Aware Optimizations" (news summary, section on the
+three optimisations, attention-efficiency paragraphs):
+
+* partially fused softmax: `qk_stats` writes the fp32 score matrix A and the
+  per-row statistics LS = (L_i, S_i) (row max, shifted sum of exponentials);
+  `softmax_av` fuses the normalisation with the product by V;
+* FlashAttention: `flash` tiles over keys with an online softmax in one kernel.
+
+This module only marshals torch tensors (device memory and streams) into the
+C ABI of libsdattn.so; all arithmetic runs in the CUDA kernels.  There is no
+CPU fallback: calls fail if the library or a CUDA device is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+
+__all__ = ["qk_stats", "softmax_av", "flash", "partially_fused", "device_error", "a_ld", "workspace_bytes",
+           "SdattnError", "load_library"]
+
+SdattnError = _lib.SdattnError
+load_library = _lib.load
+
+_DTYPES = {torch.float16: _lib.SDATTN_F16, torch.bfloat16: _lib.SDATTN_BF16}
+_workspaces: dict[int, torch.Tensor] = {}
+
+
+def _lib_handle():
+    return _lib.load()
+
+
+def make_desc(B: int, H: int, N: int, M: int, d: int, dtype: torch.dtype, scale: float) -> _lib.Desc:
+    if dtype not in _DTYPES:
+        raise TypeError(f"dtype {dtype} not supported (float16 or bfloat16)")
+    return _lib.Desc(B, H, N, M, d, _DTYPES[dtype], float(scale))
+
+
+def _scale(scale, d):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def _check_qk(q: torch.Tensor, k: torch.Tensor):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B,H,N,d] and k [B,H,M,d]")
+    if not (q.is_cuda and k.is_cuda):
+        raise ValueError("tensors must live on a CUDA device")
+    if q.dtype != k.dtype:
+        raise TypeError("q and k must share a dtype")
+    B, H, N, d = q.shape
+    if k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}")
+    return B, H, N, k.shape[2], d
+
+
+def _contig(t: torch.Tensor) -> torch.Tensor:
+    return t if t.is_contiguous() else t.contiguous()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def a_ld(desc: _lib.Desc) -> int:
+    v = _lib_handle().sdattn_a_ld(ctypes.byref(desc))
+    if v < 0:
+        raise _lib.SdattnError("sdattn_a_ld", 1)
+    return int(v)
+
+
+def workspace_bytes(desc: _lib.Desc) -> int:
+    return int(_lib_handle().sdattn_workspace_bytes(ctypes.byref(desc)))
+
+
+def workspace(desc: _lib.Desc, device: torch.device) -> torch.Tensor:
+    """A zero-filled workspace for `desc` on `device`, cached and grown on demand.
+
+    Calls that share it must be ordered on one stream (the library leaves the
+    workspace ready for the next call when a call completes)."""
+    need = max(workspace_bytes(desc), 256)
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(idx)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _workspaces[idx] = ws
+    return ws
+
+
+def qk_stats(q: torch.Tensor, k: torch.Tensor, scale: float | None = None, out_a: torch.Tensor | None = None,
+             out_ls: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """Partially fused softmax, first kernel.
+
+    Returns (A, LS): A [B,H,N,lda] fp32 with A[..., :M] = scale * Q K^T, and
+    LS [B,H,N,2] fp32 = (row max L_i, sum_j exp(A_ij - L_i))."""
+    B, H, N, M, d = _check_qk(q, k)
+    q, k = _contig(q), _contig(k)
+    desc = make_desc(B, H, N, M, d, q.dtype, _scale(scale, d))
+    lda = a_ld(desc)
+    A = out_a if out_a is not None else torch.empty((B, H, N, lda), dtype=torch.float32, device=q.device)
+    LS = out_ls if out_ls is not None else torch.empty((B, H, N, 2), dtype=torch.float32, device=q.device)
+    if A.shape != (B, H, N, lda) or A.dtype != torch.float32 or not A.is_contiguous():
+        raise ValueError(f"out_a must be contiguous fp32 [B,H,N,{lda}]")
+    if LS.shape != (B, H, N, 2) or LS.dtype != torch.float32 or not LS.is_contiguous():
+        raise ValueError("out_ls must be contiguous fp32 [B,H,N,2]")
+    w = ws if ws is not None else workspace(desc, q.device)
+    st = _lib_handle().sdattn_qk_stats(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), A.data_ptr(),
+                                       LS.data_ptr(), w.data_ptr(), w.numel(), _stream(q.device))
+    _lib.check("sdattn_qk_stats", st)
+    return A, LS
+
+
+def softmax_av(a: torch.Tensor, ls: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+               out: torch.Tensor | None = None):
+    """Partially fused softmax, second kernel: O = (sum_j exp(A_ij - L_i) V_j) / S_i.
+
+    `a` and `ls` as returned by `qk_stats`; v [B,H,M,d]."""
+    B, H, M, d = v.shape
+    N = a.shape[2]
+    if not v.is_cuda:
+        raise ValueError("v must live on a CUDA device")
+    desc = make_desc(B, H, N, M, d, v.dtype, _scale(scale, d))
+    lda = a_ld(desc)
+    if a.shape != (B, H, N, lda) or a.dtype != torch.float32 or not a.is_contiguous():
+        raise ValueError(f"a must be contiguous fp32 [B,H,N,{lda}]")
+    if ls.shape != (B, H, N, 2) or ls.dtype != torch.float32 or not ls.is_contiguous():
+        raise ValueError("ls must be contiguous fp32 [B,H,N,2]")
+    v = _contig(v)
+    O = out if out is not None else torch.empty((B, H, N, d), dtype=v.dtype, device=v.device)
+    st = _lib_handle().sdattn_softmax_av(ctypes.byref(desc), a.data_ptr(), ls.data_ptr(), v.data_ptr(),
+                                         O.data_ptr(), None, 0, _stream(v.device))
+    _lib.check("sdattn_softmax_av", st)
+    return O
+
+
+def flash(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+          out: torch.Tensor | None = None, return_ls: bool = False, out_ls: torch.Tensor | None = None):
+    """FlashAttention form.  Returns O [B,H,N,d] (and LS [B,H,N,2] if asked)."""
+    B, H, N, M, d = _check_qk(q, k)
+    if v.shape != k.shape or v.dtype != q.dtype or not v.is_cuda:
+        raise ValueError("v must match k in shape and q in dtype")
+    q, k, v = _contig(q), _contig(k), _contig(v)
+    desc = make_desc(B, H, N, M, d, q.dtype, _scale(scale, d))
+    O = out if out is not None else torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
+    LS = None
+    if return_ls or out_ls is not None:
+        LS = out_ls if out_ls is not None else torch.empty((B, H, N, 2), dtype=torch.float32, device=q.device)
+        if LS.shape != (B, H, N, 2) or LS.dtype != torch.float32 or not LS.is_contiguous():
+            raise ValueError("out_ls must be contiguous fp32 [B,H,N,2]")
+    st = _lib_handle().sdattn_flash(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), O.data_ptr(),
+                                    LS.data_ptr() if LS is not None else None, _stream(q.device))
+    _lib.check("sdattn_flash", st)
+    return (O, LS) if (return_ls or out_ls is not None) else O
+
+
+def partially_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None):
+    """Both partially fused kernels back to back; returns O."""
+    A, LS = qk_stats(q, k, scale)
+    return softmax_av(A, LS, v, scale)
+
+
+def device_error():
+    """(status name, detail code) of the device error word; reading clears it."""
+    detail = ctypes.c_uint32(0)
+    st = _lib_handle().sdattn_device_error(ctypes.byref(detail))
+    return _lib.STATUS.get(st, st), int(detail.value)

@@ -1,0 +1,314 @@
+// qk_stats.cuh -- partially fused softmax, first kernel:
+//   A = scale * Q K^T (fp32, stored), and per-row statistics (L_i, S_i).
+//
+// "Speed Is All You Need" (news summary, section on the three optimisations,
+// partially fused softmax paragraph): a kernel maps the large matrix A to the
+// vectors L and S (an N x 2 tensor) so that no full softmax runs over A; since
+// that map has far fewer outputs than inputs, A is grouped into blocks, each
+// block is reduced, and the partial results are reduced to the final ones.
+//
+// B200 design.  One persistent CTA per SM walks work units
+// (b*H + h, 128-row tile, column split).  Inside a CTA:
+//   warp 0      TMA producer: the unit's Q tile once, then a ring of K tiles;
+//   warp 1      tcgen05 MMA issuer: S = Q K^T for one 128x128 block into one
+//               of two TMEM accumulators (double-buffered);
+//   warps 2..5  epilogue, one TMEM lane (= one query row) per thread: scales
+//               the block, reduces it to a partial (m_b, s_b) pair, merges it
+//               into the row's running pair, and streams the fp32 block to HBM
+//               through swizzled shared-memory staging and TMA stores.
+// When a row's columns are split over several units, each unit writes its
+// merged pair to the workspace and bumps an arrival counter; the unit that
+// arrives last merges all splits into LS and resets the counter (no spinning).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace sdattn {
+
+struct QKParams {
+  int N, M, BH;
+  int nrt;      // 128-row tiles per (b, h)
+  int nb;       // 128-column blocks per row
+  int nsplit;   // column splits per row tile
+  int cbs;      // column blocks per split
+  int units;    // BH * nrt * nsplit
+  float scale;
+  float* LS;          // [BH][N][2]
+  float2* part;       // [BH * nrt][128][nsplit]
+  uint32_t* tickets;  // [BH * nrt]
+};
+
+template <int D>
+struct QKCfg {
+  static constexpr int DSLABS = (D + 63) / 64;    // 64-element (128 B) column slabs of Q / K
+  static constexpr int KSTEPS = (D + 15) / 16;    // K=16 MMA steps (zero-padded past D)
+  static constexpr int SLAB = 128 * 128;          // one slab of a 128-row tile, bytes
+  static constexpr int KSTAGES = DSLABS == 1 ? 4 : (DSLABS == 2 ? 3 : 2);
+  static constexpr int NSTG = 4;                  // 4 KB staging buffers per epilogue warp
+  static constexpr int STG = 4096;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + DSLABS * SLAB;
+  static constexpr int OFF_STG = OFF_K + KSTAGES * DSLABS * SLAB;
+  static constexpr int OFF_BAR = OFF_STG + 4 * NSTG * STG;
+  static constexpr int NBAR = 2 + 2 * KSTAGES + 4 + 1;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;   // + misc words + alignment slack
+  static constexpr int NTHREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 256;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void qk_decode(const QKParams& p, int u, int& bh, int& rt, int& sp, int& cb0,
+                                          int& cb1) {
+  sp = u % p.nsplit;
+  const int t = u / p.nsplit;
+  rt = t % p.nrt;
+  bh = t / p.nrt;
+  cb0 = sp * p.cbs;
+  cb1 = min(p.nb, cb0 + p.cbs);
+}
+
+// Merge of two (max, sum-of-exp) pairs: the pair of the union of their columns.
+__device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2) {
+  constexpr float L2E = 1.4426950408889634f;
+  if (m2 > m) {
+    s = s * ex2_approx((m - m2) * L2E) + s2;
+    m = m2;
+  } else {
+    s = s + s2 * ex2_approx((m2 - m) * L2E);
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(192, 1)
+    qk_stats_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmA, const QKParams p) {
+  using C = QKCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sStg = smem + C::OFF_STG;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + C::KSTAGES;
+  uint64_t* acc_full = k_empty + C::KSTAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain_bar = acc_empty + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);   // [0] tmem base, [1] abort, [2] last-split flag
+  volatile uint32_t* abort_flag = misc + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < C::KSTAGES; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(drain_bar, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmA);
+  }
+  if (warp == 1) {
+    tmem_alloc(&misc[0], C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      uint32_t kc = 0, nq = 0;   // K tiles and Q tiles issued
+      bool live = true;
+      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
+        int bh, rt, sp, cb0, cb1;
+        qk_decode(p, u, bh, rt, sp, cb0, cb1);
+        if (!mbar_wait(q_empty, (nq & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
+        ++nq;
+        mbar_arrive_expect_tx(q_full, C::DSLABS * C::SLAB);
+        for (int s = 0; s < C::DSLABS; ++s) tma_load_3d(sQ + s * C::SLAB, &tmQ, 64 * s, rt * 128, bh, q_full);
+        for (int cb = cb0; cb < cb1; ++cb, ++kc) {
+          const uint32_t st = kc % C::KSTAGES, n = kc / C::KSTAGES;
+          if (!mbar_wait(&k_empty[st], (n & 1) ^ 1, kSiteKEmpty, abort_flag)) { live = false; break; }
+          mbar_arrive_expect_tx(&k_full[st], C::DSLABS * C::SLAB);
+          for (int s = 0; s < C::DSLABS; ++s)
+            tma_load_3d(sK + (st * C::DSLABS + s) * C::SLAB, &tmK, 64 * s, cb * 128, bh, &k_full[st]);
+        }
+      }
+      // Let every load this thread issued land before the CTA can exit.
+      volatile uint32_t never = 0;
+      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, kSiteQFull, &never);
+      for (uint32_t st = 0; st < C::KSTAGES && st < kc; ++st) {
+        const uint32_t uses = (kc - st + C::KSTAGES - 1) / C::KSTAGES;
+        mbar_wait(&k_full[st], (uses - 1) & 1, kSiteKFull, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer --------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, 128, BF16, false, false);
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
+      uint32_t kc = 0, ac = 0, ui = 0;
+      bool live = true;
+      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
+        int bh, rt, sp, cb0, cb1;
+        qk_decode(p, u, bh, rt, sp, cb0, cb1);
+        if (!mbar_wait(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
+        tc_fence_after();
+        for (int cb = cb0; cb < cb1; ++cb, ++kc, ++ac) {
+          const uint32_t st = kc % C::KSTAGES, n = kc / C::KSTAGES;
+          const uint32_t ab = ac & 1, na = ac >> 1;
+          if (!mbar_wait(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait(&acc_empty[ab], (na & 1) ^ 1, kSiteAccEmpty, abort_flag)) { live = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + ab * 128;
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint32_t off = (kk >> 2) * C::SLAB + (kk & 3) * 32;
+            const uint64_t ad = sdesc_sw128(q_base + off, 16, 1024);
+            const uint64_t bd = sdesc_sw128(k_base + st * C::DSLABS * C::SLAB + off, 16, 1024);
+            mma_ss(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&k_empty[st]);
+          mma_commit(&acc_full[ab]);
+        }
+        if (live) mma_commit(q_empty);
+      }
+      // Wait until every MMA this thread issued has finished.
+      volatile uint32_t never = 0;
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, kSiteAccFull, &never);
+    }
+  } else {
+    // ------------------------------ epilogue ----------------------------------
+    constexpr float L2E = 1.4426950408889634f;
+    const int quarter = warp & 3;                 // TMEM lanes quarter*32 .. +31
+    const int row_local = quarter * 32 + lane;    // row of the 128-row tile
+    uint8_t* stg = sStg + (warp - 2) * C::NSTG * C::STG;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t ac = 0, sc = 0;
+    bool live = true;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+      int bh, rt, sp, cb0, cb1;
+      qk_decode(p, u, bh, rt, sp, cb0, cb1);
+      float m_run = -INFINITY, s_run = 0.f;
+      for (int cb = cb0; cb < cb1 && live; ++cb, ++ac) {
+        const uint32_t ab = ac & 1, na = ac >> 1;
+        live = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], na & 1, kSiteAccFull, abort_flag));
+        if (!live) break;
+        tc_fence_after();
+        uint32_t v[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_x32(tmem + ab * 128 + c * 32 + lane_off, v + 32 * c);
+        tmem_wait_ld();
+        reg_fence<128>(v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+
+        float a[128];
+#pragma unroll
+        for (int k = 0; k < 128; ++k) a[k] = __uint_as_float(v[k]) * p.scale;
+        const int col0 = cb * 128;
+        const int valid = min(128, p.M - col0);
+        // block partial (m_b, s_b) over the valid columns of this 128-column block
+        float mb = -INFINITY;
+        float sb = 0.f;
+        if (valid == 128) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) mb = fmaxf(mb, a[k]);
+          const float nmb = -mb * L2E;
+#pragma unroll
+          for (int k = 0; k < 128; ++k) sb += ex2_approx(fmaf(a[k], L2E, nmb));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) mb = (k < valid) ? fmaxf(mb, a[k]) : mb;
+          const float nmb = -mb * L2E;
+#pragma unroll
+          for (int k = 0; k < 128; ++k) sb += (k < valid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
+        }
+        ms_merge(m_run, s_run, mb, sb);
+
+        // stream the block to A: 4 chunks of 32 columns x this warp's 32 rows
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (col0 + 32 * c >= p.M) break;
+          uint8_t* buf = stg + (sc % C::NSTG) * C::STG;
+          if (lane == 0) bulk_wait_read<C::NSTG - 1>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 w = make_float4(a[32 * c + 4 * j + 0], a[32 * c + 4 * j + 1], a[32 * c + 4 * j + 2],
+                                   a[32 * c + 4 * j + 3]);
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmA, buf, col0 + 32 * c, rt * 128 + quarter * 32, bh);
+            bulk_commit();
+          }
+          ++sc;
+        }
+      }
+      // ---- unit result: the merged pair of this split ----
+      const int row = rt * 128 + row_local;
+      if (p.nsplit == 1) {
+        if (live && row < p.N)
+          *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(m_run, s_run);
+      } else {
+        const int64_t tile = static_cast<int64_t>(bh) * p.nrt + rt;
+        if (live) p.part[(tile * 128 + row_local) * p.nsplit + sp] = make_float2(m_run, s_run);
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          uint32_t last = 0;
+          if (live) {
+            __threadfence();
+            last = (atomicAdd(&p.tickets[tile], 1u) == static_cast<uint32_t>(p.nsplit - 1)) ? 1u : 0u;
+          }
+          misc[2] = last;
+        }
+        named_bar_sync(1, 128);
+        if (misc[2]) {
+          __threadfence();
+          float m = -INFINITY, s = 0.f;
+          const float2* pr = p.part + (tile * 128 + row_local) * p.nsplit;
+          for (int k = 0; k < p.nsplit; ++k) {
+            const float2 q = __ldcg(pr + k);
+            ms_merge(m, s, q.x, q.y);
+          }
+          if (row < p.N)
+            *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(m, s);
+          if (threadIdx.x == 64) p.tickets[tile] = 0u;
+        }
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace sdattn

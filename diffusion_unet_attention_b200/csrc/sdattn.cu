@@ -1,0 +1,376 @@
+// sdattn.cu -- host side of libsdattn: argument checks, TMA tensor maps,
+// work partitioning and launches of the sm_100a kernels.  Every entry point is
+// declared (and documented) in include/sdattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "sdattn.h"
+
+#include "flash.cuh"
+#include "qk_stats.cuh"
+#include "softmax_av.cuh"
+
+namespace {
+
+using sdattn::AVCfg;
+using sdattn::AVParams;
+using sdattn::FlashCfg;
+using sdattn::FlashParams;
+using sdattn::QKCfg;
+using sdattn::QKParams;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSplit = 16;
+
+// --------------------------------------------------------------------------
+// Driver entry point for tensor-map encoding (no link-time libcuda dependency)
+// --------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D tiled map: dims {d0 (contiguous), d1, d2}, byte strides of d1 and d2,
+// box {b0, b1, 1}, 128-byte swizzle, zero fill outside the tensor.
+bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------------------
+// Device facts
+// --------------------------------------------------------------------------
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int sm_count(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename Kern>
+bool ensure_smem(Kern kern, int bytes, std::atomic<uint64_t>& done, int dev) {
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+// --------------------------------------------------------------------------
+// Validation
+// --------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sdattn_status check_desc(const sdattn_desc* d) {
+  if (!d) return SDATTN_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->N < 1 || d->M < 1) return SDATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(d->scale) || !(d->scale > 0.f)) return SDATTN_ERR_INVALID_ARG;
+  if (d->d != 40 && d->d != 80 && d->d != 160) return SDATTN_ERR_UNSUPPORTED;
+  if (d->dtype != SDATTN_F16 && d->dtype != SDATTN_BF16) return SDATTN_ERR_UNSUPPORTED;
+  const int64_t bh = static_cast<int64_t>(d->B) * d->H;
+  if (bh * d->N >= (int64_t(1) << 31) || bh * d->M >= (int64_t(1) << 31)) return SDATTN_ERR_UNSUPPORTED;
+  if (bh >= (int64_t(1) << 31)) return SDATTN_ERR_UNSUPPORTED;
+  return SDATTN_OK;
+}
+
+int64_t a_ld(const sdattn_desc* d) { return (static_cast<int64_t>(d->M) + 3) / 4 * 4; }
+
+CUtensorMapDataType elem_type(const sdattn_desc* d) {
+  return d->dtype == SDATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
+// Column splits of the statistics reduction: the smallest power of two that
+// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit.
+struct QKPlan {
+  int nrt, nb, nsplit, cbs, units;
+};
+
+QKPlan plan_qk(const sdattn_desc* d, int nsm) {
+  QKPlan pl;
+  const int bh = d->B * d->H;
+  pl.nrt = (d->N + 127) / 128;
+  pl.nb = (d->M + 127) / 128;
+  const int64_t base = static_cast<int64_t>(bh) * pl.nrt;
+  auto eff = [&](int64_t u) {
+    const int64_t waves = (u + nsm - 1) / nsm;
+    return static_cast<double>(u) / static_cast<double>(waves * nsm);
+  };
+  int ns = 1;
+  const int cap = pl.nb < kMaxSplit ? pl.nb : kMaxSplit;
+  while (ns * 2 <= cap && eff(base * ns) < 0.9) ns *= 2;
+  pl.cbs = (pl.nb + ns - 1) / ns;
+  pl.nsplit = (pl.nb + pl.cbs - 1) / pl.cbs;
+  pl.units = static_cast<int>(base * pl.nsplit);
+  return pl;
+}
+
+// Workspace: [tickets: one uint32 per (b, h, row tile), padded to 256 B]
+//            [partials: float2 per (b, h, row tile, row, split)]
+size_t ws_tickets_bytes(const sdattn_desc* d) {
+  const int64_t tiles = static_cast<int64_t>(d->B) * d->H * ((d->N + 127) / 128);
+  return static_cast<size_t>((tiles * 4 + 255) / 256 * 256);
+}
+
+size_t ws_bytes(const sdattn_desc* d) {
+  const int64_t tiles = static_cast<int64_t>(d->B) * d->H * ((d->N + 127) / 128);
+  const int nb = (d->M + 127) / 128;
+  const int smax = nb < kMaxSplit ? nb : kMaxSplit;
+  return ws_tickets_bytes(d) + static_cast<size_t>(tiles) * 128 * smax * sizeof(float2);
+}
+
+// --------------------------------------------------------------------------
+// Launchers
+// --------------------------------------------------------------------------
+template <int D, bool BF16>
+sdattn_status launch_qk(const sdattn_desc* d, const void* Q, const void* K, float* A, float* LS, void* ws,
+                        cudaStream_t stream) {
+  using C = QKCfg<D>;
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  auto kern = sdattn::qk_stats_kernel<D, BF16>;
+  static std::atomic<uint64_t> smem_done{0};
+  if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
+
+  const int nsm = sm_count(dev);
+  const QKPlan pl = plan_qk(d, nsm);
+  const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
+  const uint64_t N = d->N, M = d->M, lda = a_ld(d);
+  CUtensorMap mq, mk, ma;
+  if (!make_map_3d(&mq, Q, elem_type(d), D, N, bh, D * 2, N * D * 2, 64, 128)) return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&mk, K, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, 128)) return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, N, bh, lda * 4, N * lda * 4, 32, 32))
+    return SDATTN_ERR_CUDA;
+
+  QKParams p;
+  p.N = d->N;
+  p.M = d->M;
+  p.BH = static_cast<int>(bh);
+  p.nrt = pl.nrt;
+  p.nb = pl.nb;
+  p.nsplit = pl.nsplit;
+  p.cbs = pl.cbs;
+  p.units = pl.units;
+  p.scale = d->scale;
+  p.LS = LS;
+  p.tickets = static_cast<uint32_t*>(ws);
+  p.part = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + ws_tickets_bytes(d));
+  const int grid = pl.units < nsm ? pl.units : nsm;
+  kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, ma, p);
+  return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+sdattn_status launch_av(const sdattn_desc* d, const float* A, const float* LS, const void* V, void* O,
+                        cudaStream_t stream) {
+  using C = AVCfg<D>;
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  auto kern = sdattn::softmax_av_kernel<D, BF16>;
+  static std::atomic<uint64_t> smem_done{0};
+  if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
+
+  const int nsm = sm_count(dev);
+  const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
+  const uint64_t N = d->N, M = d->M, lda = a_ld(d);
+  CUtensorMap ma, mv;
+  if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, N, bh, lda * 4, N * lda * 4, 32, 128))
+    return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&mv, V, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, C::BK)) return SDATTN_ERR_CUDA;
+
+  AVParams p;
+  p.N = d->N;
+  p.M = d->M;
+  p.BH = static_cast<int>(bh);
+  p.nrt = (d->N + 127) / 128;
+  p.nkb = (d->M + C::BK - 1) / C::BK;
+  p.units = p.BH * p.nrt;
+  p.LS = LS;
+  p.O = O;
+  const int grid = p.units < nsm ? p.units : nsm;
+  kern<<<grid, 192, C::SMEM, stream>>>(ma, mv, p);
+  return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
+}
+
+template <int D, int NQ, int BN, bool BF16>
+sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
+                           cudaStream_t stream) {
+  using C = FlashCfg<D, NQ, BN>;
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  auto kern = sdattn::flash_kernel<D, NQ, BN, BF16>;
+  static std::atomic<uint64_t> smem_done{0};
+  if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
+
+  const int nsm = sm_count(dev);
+  const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
+  const uint64_t N = d->N, M = d->M;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_3d(&mq, Q, elem_type(d), D, N, bh, D * 2, N * D * 2, 64, 128)) return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&mk, K, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, BN)) return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&mv, V, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, BN)) return SDATTN_ERR_CUDA;
+
+  FlashParams p;
+  p.N = d->N;
+  p.M = d->M;
+  p.BH = static_cast<int>(bh);
+  p.tph = (d->N + 128 * NQ - 1) / (128 * NQ);
+  p.nkv = (d->M + BN - 1) / BN;
+  p.units = p.BH * p.tph;
+  p.scale = d->scale;
+  p.c = d->scale * 1.4426950408889634f;
+  p.O = O;
+  p.LS = LS;
+  const int grid = p.units < nsm ? p.units : nsm;
+  kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
+}
+
+template <bool BF16>
+sdattn_status dispatch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
+                             cudaStream_t s) {
+  const int dev = current_device();
+  const int nsm = sm_count(dev < 0 ? 0 : dev);
+  const int64_t pairs = static_cast<int64_t>(d->B) * d->H * ((d->N + 255) / 256);
+  const bool two = pairs >= nsm;   // enough work for two query tiles per CTA
+  switch (d->d) {
+    case 40:
+      return two ? launch_flash<40, 2, 128, BF16>(d, Q, K, V, O, LS, s)
+                 : launch_flash<40, 1, 128, BF16>(d, Q, K, V, O, LS, s);
+    case 80:
+      return two ? launch_flash<80, 2, 128, BF16>(d, Q, K, V, O, LS, s)
+                 : launch_flash<80, 1, 128, BF16>(d, Q, K, V, O, LS, s);
+    case 160:
+      return launch_flash<160, 1, 64, BF16>(d, Q, K, V, O, LS, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+int64_t sdattn_a_ld(const sdattn_desc* desc) {
+  if (check_desc(desc) != SDATTN_OK) return -1;
+  return a_ld(desc);
+}
+
+size_t sdattn_workspace_bytes(const sdattn_desc* desc) {
+  if (check_desc(desc) != SDATTN_OK) return 0;
+  return ws_bytes(desc);
+}
+
+sdattn_status sdattn_qk_stats(const sdattn_desc* desc, const void* Q, const void* K, float* A, float* LS, void* ws,
+                              size_t ws_size, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !A || !LS) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(A) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
+  if (!ws || ws_size < ws_bytes(desc)) return SDATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf = desc->dtype == SDATTN_BF16;
+  switch (desc->d) {
+    case 40: return bf ? launch_qk<40, true>(desc, Q, K, A, LS, ws, s) : launch_qk<40, false>(desc, Q, K, A, LS, ws, s);
+    case 80: return bf ? launch_qk<80, true>(desc, Q, K, A, LS, ws, s) : launch_qk<80, false>(desc, Q, K, A, LS, ws, s);
+    case 160:
+      return bf ? launch_qk<160, true>(desc, Q, K, A, LS, ws, s) : launch_qk<160, false>(desc, Q, K, A, LS, ws, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
+}
+
+sdattn_status sdattn_softmax_av(const sdattn_desc* desc, const float* A, const float* LS, const void* V, void* O,
+                                void* ws, size_t ws_size, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!A || !LS || !V || !O) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(LS) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
+  if (ws && !aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
+  if (!ws && ws_size != 0) return SDATTN_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf = desc->dtype == SDATTN_BF16;
+  switch (desc->d) {
+    case 40: return bf ? launch_av<40, true>(desc, A, LS, V, O, s) : launch_av<40, false>(desc, A, LS, V, O, s);
+    case 80: return bf ? launch_av<80, true>(desc, A, LS, V, O, s) : launch_av<80, false>(desc, A, LS, V, O, s);
+    case 160: return bf ? launch_av<160, true>(desc, A, LS, V, O, s) : launch_av<160, false>(desc, A, LS, V, O, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
+}
+
+sdattn_status sdattn_flash(const sdattn_desc* desc, const void* Q, const void* K, const void* V, void* O,
+                           float* LS_or_null, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !V || !O) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
+  if (LS_or_null && !aligned16(LS_or_null)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return desc->dtype == SDATTN_BF16 ? dispatch_flash<true>(desc, Q, K, V, O, LS_or_null, s)
+                                    : dispatch_flash<false>(desc, Q, K, V, O, LS_or_null, s);
+}
+
+sdattn_status sdattn_device_error(uint32_t* detail) {
+  if (detail) *detail = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SDATTN_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, sdattn::g_error_word, sizeof(v)) != cudaSuccess) return SDATTN_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(sdattn::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SDATTN_ERR_CUDA;
+  if (detail) *detail = v;
+  return v ? SDATTN_ERR_TIMEOUT : SDATTN_OK;
+}
+
+const char* sdattn_status_string(sdattn_status status) {
+  switch (status) {
+    case SDATTN_OK: return "ok";
+    case SDATTN_ERR_INVALID_ARG: return "invalid argument";
+    case SDATTN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case SDATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case SDATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case SDATTN_ERR_CUDA: return "CUDA runtime or driver error";
+    case SDATTN_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t sdattn_version(void) { return 100; }
+
+}  // extern "C"

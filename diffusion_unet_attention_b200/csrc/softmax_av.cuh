@@ -1,0 +1,256 @@
+// softmax_av.cuh -- partially fused softmax, second kernel: the softmax
+// normalisation fused with the multiplication by V,
+//   O_i = (sum_j exp(A_ij - L_i) V_j) / S_i.
+//
+// "Speed Is All You Need" (news summary, section on the three optimisations,
+// partially fused softmax paragraph): once L and S are known, the softmax is
+// fused with the matrix multiplication by V, so no normalised probability
+// matrix is ever written.
+//
+// B200 design.  One persistent CTA per SM walks (b*H + h, 128-row tile) units.
+//   warp 0      TMA producer: a ring of (A block 128 x 64 fp32, V block 64 x d)
+//               stages, 128-byte swizzled;
+//   warps 2..5  one query row per thread: reads its 64 scores of the block from
+//               shared memory, computes p = exp(a - L_i) in registers, packs p
+//               to 16 bits and writes it to tensor memory (double-buffered);
+//   warp 1      tcgen05 MMA issuer: O += P V with P taken from tensor memory
+//               and V from shared memory, O accumulated in tensor memory.
+// The epilogue scales O by 1/S_i and stores it.  Since L_i is final, no
+// rescaling is ever needed.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace sdattn {
+
+struct AVParams {
+  int N, M, BH;
+  int nrt;    // 128-row tiles per (b, h)
+  int nkb;    // 64-key blocks
+  int units;  // BH * nrt
+  const float* LS;
+  void* O;
+};
+
+template <int D>
+struct AVCfg {
+  static constexpr int DSLABS = (D + 63) / 64;
+  static constexpr int PVN = DSLABS * 64;              // MMA N (head width padded to 64)
+  static constexpr int BK = 64;                        // keys per block
+  static constexpr int A_BYTES = 128 * BK * 4;         // 32 KB: two 16 KB boxes of 32 fp32 columns
+  static constexpr int V_SLAB = BK * 128;              // 8 KB: 64 keys x 64 elements
+  static constexpr int V_BYTES = DSLABS * V_SLAB;
+  static constexpr int STAGES = D == 160 ? 3 : 4;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_V = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * V_BYTES;
+  static constexpr int NBAR = 4 * STAGES + 4 + 1 + 1;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t TM_P = 0;      // two P buffers of 32 columns (128 x 64 16-bit)
+  static constexpr uint32_t TM_O = 64;     // O accumulator, PVN columns
+  static_assert(TM_O + PVN <= TMEM_COLS, "tensor memory budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(192, 1)
+    softmax_av_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
+                      const AVParams p) {
+  using C = AVCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sV = smem + C::OFF_V;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = a_full + C::STAGES;
+  uint64_t* v_full = a_empty + C::STAGES;
+  uint64_t* v_empty = v_full + C::STAGES;
+  uint64_t* p_full = v_empty + C::STAGES;
+  uint64_t* p_empty = p_full + 2;
+  uint64_t* o_full = p_empty + 2;
+  uint64_t* drain_bar = o_full + 1;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile uint32_t* abort_flag = misc + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 4);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_empty[i], 1);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(drain_bar, 1);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&misc[0], C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      uint32_t c = 0;
+      bool live = true;
+      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
+        const int bh = u / p.nrt, rt = u % p.nrt;
+        for (int kb = 0; kb < p.nkb; ++kb, ++c) {
+          const uint32_t st = c % C::STAGES, n = c / C::STAGES;
+          if (!mbar_wait(&a_empty[st], (n & 1) ^ 1, kSiteAEmpty, abort_flag)) { live = false; break; }
+          if (!mbar_wait(&v_empty[st], (n & 1) ^ 1, kSiteVEmpty, abort_flag)) { live = false; break; }
+          mbar_arrive_expect_tx(&a_full[st], C::A_BYTES);
+          tma_load_3d(sA + st * C::A_BYTES, &tmA, kb * C::BK, rt * 128, bh, &a_full[st]);
+          tma_load_3d(sA + st * C::A_BYTES + C::A_BYTES / 2, &tmA, kb * C::BK + 32, rt * 128, bh, &a_full[st]);
+          mbar_arrive_expect_tx(&v_full[st], C::V_BYTES);
+          for (int s = 0; s < C::DSLABS; ++s)
+            tma_load_3d(sV + st * C::V_BYTES + s * C::V_SLAB, &tmV, 64 * s, kb * C::BK, bh, &v_full[st]);
+        }
+      }
+      volatile uint32_t never = 0;
+      for (uint32_t st = 0; st < C::STAGES && st < c; ++st) {
+        const uint32_t uses = (c - st + C::STAGES - 1) / C::STAGES;
+        mbar_wait(&a_full[st], (uses - 1) & 1, kSiteAFull, &never);
+        mbar_wait(&v_full[st], (uses - 1) & 1, kSiteVFull, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer --------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, C::PVN, BF16, false, true);
+      const uint32_t v_base = smem_u32(sV);
+      uint32_t c = 0, pc = 0;
+      bool live = true;
+      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
+        for (int kb = 0; kb < p.nkb; ++kb, ++c, ++pc) {
+          const uint32_t st = c % C::STAGES, n = c / C::STAGES;
+          const uint32_t pb = pc & 1, np = pc >> 1;
+          if (!mbar_wait(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait(&p_full[pb], np & 1, kSitePFull, abort_flag)) { live = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            // V block, MN-major: 16 keys = two 8-row groups (SBO 1024 B apart);
+            // 64-element column slabs C::V_SLAB bytes apart (LBO).
+            const uint64_t bd = sdesc_sw128(v_base + st * C::V_BYTES + kk * 2048, C::V_SLAB, 1024);
+            mma_ts(tmem + C::TM_O, tmem + C::TM_P + pb * 32 + kk * 8, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&v_empty[st]);
+          mma_commit(&p_empty[pb]);
+        }
+        if (live) mma_commit(o_full);
+      }
+      volatile uint32_t never = 0;
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, kSiteOFull, &never);
+    }
+  } else {
+    // --------------------- softmax rows and epilogue --------------------------
+    constexpr float L2E = 1.4426950408889634f;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                // row of the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t c = 0, pc = 0, ui = 0;
+    bool live = true;
+    for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
+      const int bh = u / p.nrt, rt = u % p.nrt;
+      const int row = rt * 128 + r;
+      float Lr = 0.f, Sr = 1.f;
+      if (row < p.N) {
+        const float2 ls = *reinterpret_cast<const float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row));
+        Lr = ls.x;
+        Sr = ls.y;
+      }
+      const float nl = -Lr * L2E;
+      for (int kb = 0; kb < p.nkb; ++kb, ++c, ++pc) {
+        const uint32_t st = c % C::STAGES, n = c / C::STAGES;
+        live = __all_sync(0xffffffffu, mbar_wait(&a_full[st], n & 1, kSiteAFull, abort_flag));
+        if (!live) break;
+        // this row's 64 scores: two 32-column boxes, 128-byte swizzled rows
+        uint32_t pk[32];
+        const int valid = p.M - kb * C::BK;           // columns of this block inside [0, M)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint8_t* rowp = sA + st * C::A_BYTES + h * (C::A_BYTES / 2) + r * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 a = *reinterpret_cast<const float4*>(rowp + ((j ^ (r & 7)) << 4));
+            const int k = h * 32 + 4 * j;
+            float e0 = ex2_approx(fmaf(a.x, L2E, nl));
+            float e1 = ex2_approx(fmaf(a.y, L2E, nl));
+            float e2 = ex2_approx(fmaf(a.z, L2E, nl));
+            float e3 = ex2_approx(fmaf(a.w, L2E, nl));
+            if (valid < C::BK) {
+              e0 = (k + 0 < valid) ? e0 : 0.f;
+              e1 = (k + 1 < valid) ? e1 : 0.f;
+              e2 = (k + 2 < valid) ? e2 : 0.f;
+              e3 = (k + 3 < valid) ? e3 : 0.f;
+            }
+            pk[k / 2 + 0] = pack2<BF16>(e0, e1);
+            pk[k / 2 + 1] = pack2<BF16>(e2, e3);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_empty[st]);
+        const uint32_t pb = pc & 1, np = pc >> 1;
+        live = __all_sync(0xffffffffu, mbar_wait(&p_empty[pb], (np & 1) ^ 1, kSitePEmpty, abort_flag));
+        if (!live) break;
+        tc_fence_after();
+        tmem_st_x16(tmem + C::TM_P + pb * 32 + lane_off, pk);
+        tmem_st_x16(tmem + C::TM_P + pb * 32 + 16 + lane_off, pk + 16);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[pb]);
+      }
+      if (!live) break;
+      // ---- epilogue: O_i / S_i ----
+      live = __all_sync(0xffffffffu, mbar_wait(o_full, ui & 1, kSiteOFull, abort_flag));
+      if (!live) break;
+      tc_fence_after();
+      const float inv = 1.f / Sr;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row) * D * 2;
+#pragma unroll
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        uint32_t o[8];
+        tmem_ld_x8(tmem + C::TM_O + c8 * 8 + lane_off, o);
+        tmem_wait_ld();
+        reg_fence<8>(o);
+        uint4 w;
+        w.x = pack2<BF16>(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+        w.y = pack2<BF16>(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+        w.z = pack2<BF16>(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+        w.w = pack2<BF16>(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+        if (row < p.N) *reinterpret_cast<uint4*>(orow + c8 * 16) = w;
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace sdattn

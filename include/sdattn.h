@@ -1,0 +1,143 @@
+/*
+ * sdattn.h -- C ABI of libsdattn, B200 (sm_100a) attention for the
+ * transformer blocks of Stable Diffusion's UNet:  O = softmax(scale Q K^T) V.
+ *
+ * Source of the method: "Speed Is All You Need: On-Device Acceleration of
+ * Large Diffusion Models via GPU-Aware Optimizations" (Chen et al., CVPR
+ * Workshops 2023), as summarised in the news page on m.danchuang.com.cn,
+ * section on the three optimisations ("improving attention efficiency").
+ * That section describes two forms of attention:
+ *
+ *   1. Partially fused softmax.  Instead of running a full softmax over the
+ *      large score matrix A, one kernel reduces A to per-row vectors L and S
+ *      (an N x 2 tensor), the reduction split over blocks of A with the
+ *      partial results reduced to the final ones; a second kernel fuses the
+ *      softmax normalisation with the multiplication by V.
+ *      -> sdattn_qk_stats, sdattn_softmax_av
+ *   2. FlashAttention: exact attention computed tile by tile in one kernel
+ *      without writing A to memory.
+ *      -> sdattn_flash
+ *
+ * The page gives no formula for L and S.  This library reads them as
+ *      L_i = max_j A_ij,     S_i = sum_j exp(A_ij - L_i)      (natural base)
+ * with A = scale * Q K^T, so that softmax(A)_ij = exp(A_ij - L_i) / S_i.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensors are caller-owned DEVICE buffers, row-major and contiguous:
+ *        Q  [B][H][N][d]      element type desc->dtype
+ *        K  [B][H][M][d]      element type desc->dtype
+ *        V  [B][H][M][d]      element type desc->dtype
+ *        O  [B][H][N][d]      element type desc->dtype
+ *        A  [B][H][N][lda]    float32, lda = sdattn_a_ld(desc) >= M; only the
+ *                             first M entries of each row are read or written
+ *        LS [B][H][N][2]      float32, (L_i, S_i) pairs
+ *  - Every pointer must be 16-byte aligned.  Buffers must not overlap.
+ *  - Calls only enqueue work on `stream` (a cudaStream_t, or NULL for the
+ *    legacy default stream) and return; results are ready when the stream
+ *    reaches them.  Argument errors are detected on the host before anything
+ *    is enqueued and nothing is written.  The library allocates no memory,
+ *    never calls exit/abort/__trap, and lets no C++ exception cross the ABI.
+ *  - The library keeps one device-resident error word per device.  A kernel
+ *    whose internal wait exceeds its time limit (about one second) records
+ *    SDATTN_ERR_TIMEOUT there and returns early; sdattn_device_error() reads
+ *    and clears it.
+ *  - Supported: d in {40, 80, 160} (the UNet's head widths), dtype F16 or
+ *    BF16, B*H*N and B*H*M below 2^31, M and N at least 1, scale > 0.
+ *  - Thread safety: calls on different streams may run concurrently; calls
+ *    that share a workspace must be ordered on one stream.
+ */
+#ifndef SDATTN_H
+#define SDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SDATTN_F16 = 0,   /* IEEE binary16 */
+    SDATTN_BF16 = 1   /* bfloat16 */
+} sdattn_dtype;
+
+/* Shape of one attention call.  scale is applied to Q K^T (1/sqrt(d) in SD). */
+typedef struct {
+    int32_t B;        /* batch (2 for a classifier-free-guidance pair) */
+    int32_t H;        /* heads */
+    int32_t N;        /* query rows per (b, h) */
+    int32_t M;        /* key / value rows per (b, h) */
+    int32_t d;        /* head width: 40, 80 or 160 */
+    int32_t dtype;    /* sdattn_dtype of Q, K, V and O */
+    float scale;      /* finite, positive score scale */
+} sdattn_desc;
+
+typedef enum {
+    SDATTN_OK = 0,
+    SDATTN_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, scale not finite and > 0 */
+    SDATTN_ERR_UNSUPPORTED = 2,   /* d or dtype outside the supported set */
+    SDATTN_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    SDATTN_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    SDATTN_ERR_CUDA = 5,          /* a CUDA runtime / driver call failed */
+    SDATTN_ERR_TIMEOUT = 6        /* a kernel's bounded wait ran out (device error word) */
+} sdattn_status;
+
+/* Row stride of A in floats: M rounded up to a multiple of 4 (16-byte rows).
+ * Returns -1 for an invalid descriptor. */
+int64_t sdattn_a_ld(const sdattn_desc *desc);
+
+/* Bytes of workspace that sdattn_qk_stats and sdattn_softmax_av need for this
+ * shape on the current device (split-reduction partials plus arrival
+ * counters).  The same workspace serves both calls.  It must be zero-filled
+ * once before its first use; every completed call leaves it ready for the next
+ * (its counters back at zero).  Returns 0 for an invalid descriptor. */
+size_t sdattn_workspace_bytes(const sdattn_desc *desc);
+
+/* Partially fused softmax, first kernel: the score matrix and its row
+ * statistics, in one launch.
+ *   A[b][h][i][j] = scale * sum_k Q[b][h][i][k] K[b][h][j][k]   (fp32, j < M)
+ *   LS[b][h][i]   = (L_i, S_i) as defined above.
+ * The reduction follows the page's split: each 128-column block of a row is
+ * reduced to a partial (m, s) pair, partial pairs are merged per column split,
+ * and the last split to finish merges the splits into LS.
+ * Q, K: inputs; A, LS: outputs; ws: workspace of ws_bytes >=
+ * sdattn_workspace_bytes(desc) bytes, zero-filled before first use. */
+sdattn_status sdattn_qk_stats(const sdattn_desc *desc, const void *Q, const void *K,
+                              float *A, float *LS, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/* Partially fused softmax, second kernel: normalisation fused with the
+ * multiplication by V.
+ *   O[b][h][i][c] = (sum_j exp(A_ij - L_i) V[b][h][j][c]) / S_i
+ * A, LS (as written by sdattn_qk_stats), V: inputs; O: output.
+ * ws / ws_bytes: optional workspace (may be NULL / 0); when given (at least
+ * sdattn_workspace_bytes(desc) bytes, zero-filled before first use) the key
+ * range may be split across CTAs for small problems. */
+sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const float *LS,
+                                const void *V, void *O, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* FlashAttention form: one kernel, tiled over keys with an online softmax,
+ * A never stored.  Q, K, V: inputs; O: output.  LS_or_null: if not NULL,
+ * also receives (L_i, S_i) as defined above. */
+sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K,
+                           const void *V, void *O, float *LS_or_null, void *stream);
+
+/* Reads and clears this device's error word (synchronises the device).
+ * Returns SDATTN_OK, SDATTN_ERR_TIMEOUT, or SDATTN_ERR_CUDA if it cannot be
+ * read.  If detail is not NULL it receives a code naming the wait that ran
+ * out (0 when none). */
+sdattn_status sdattn_device_error(uint32_t *detail);
+
+/* Static, human-readable name of a status. */
+const char *sdattn_status_string(sdattn_status status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int32_t sdattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDATTN_H */

@@ -1,0 +1,91 @@
+"""The C ABI library loads, exports what include/sdattn.h declares, and rejects
+bad arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from diffusion_unet_attention_b200 import _lib, build
+    build.build()
+    return _lib.load()
+
+
+def _desc(B=2, H=8, N=4096, M=4096, d=40, dtype=0, scale=0.158113883):
+    from diffusion_unet_attention_b200 import _lib
+    return _lib.Desc(B, H, N, M, d, dtype, scale)
+
+
+def test_header_declarations_are_exported(lib):
+    from diffusion_unet_attention_b200 import _lib
+    hdr = open(os.path.join(ROOT, "include", "sdattn.h")).read()
+    declared = set(re.findall(r"\b(sdattn_[a-z_]+)\s*\(", hdr))
+    assert declared == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_a_ld_and_workspace(lib):
+    for M, ld in [(4096, 4096), (77, 80), (1, 4), (64, 64), (129, 132)]:
+        assert lib.sdattn_a_ld(ctypes.byref(_desc(M=M))) == ld
+    assert lib.sdattn_a_ld(ctypes.byref(_desc(d=64))) == -1
+    ws = lib.sdattn_workspace_bytes(ctypes.byref(_desc()))
+    # tickets for 2*8*32 row tiles plus 16 splits of 128 float2 per tile
+    assert ws >= 2 * 8 * 32 * 128 * 16 * 8
+    assert lib.sdattn_workspace_bytes(ctypes.byref(_desc(N=0))) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), 1), (dict(N=0), 1), (dict(M=-1), 1), (dict(scale=float("inf")), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=0.0), 1), (dict(scale=-0.1), 1), (dict(d=64), 2), (dict(d=128), 2), (dict(dtype=7), 2),
+])
+def test_bad_descriptor(lib, kw, status):
+    d = _desc(**kw)
+    p = ctypes.c_void_p(4096)
+    assert lib.sdattn_flash(ctypes.byref(d), p, p, p, p, None, None) == status
+    assert lib.sdattn_qk_stats(ctypes.byref(d), p, p, p, p, p, 1 << 30, None) == status
+    assert lib.sdattn_softmax_av(ctypes.byref(d), p, p, p, p, None, 0, None) == status
+
+
+def test_null_and_misaligned_pointers(lib):
+    d = _desc()
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.sdattn_flash(None, ok, ok, ok, ok, None, None) == 1
+    assert lib.sdattn_flash(ctypes.byref(d), None, ok, ok, ok, None, None) == 1
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, bad, ok, None, None) == 3
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, bad, None) == 3
+    assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, None, None, 0, None) == 1
+    assert lib.sdattn_softmax_av(ctypes.byref(d), bad, ok, ok, ok, None, 0, None) == 3
+    assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, bad, ok, 1 << 30, None) == 3
+
+
+def test_workspace_checked(lib):
+    d = _desc()
+    ok = ctypes.c_void_p(1 << 20)
+    need = lib.sdattn_workspace_bytes(ctypes.byref(d))
+    assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, None, need, None) == 4
+    assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, ok, need - 1, None) == 4
+    assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, ok, None, 16, None) == 4
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.sdattn_status_string(s)
+    assert lib.sdattn_status_string(99) == b"unknown status"
+    assert lib.sdattn_version() >= 100
+
+
+def test_python_api_refuses_cpu_tensors():
+    import torch
+    import diffusion_unet_attention_b200 as sd
+    q = torch.zeros(1, 1, 8, 40, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        sd.flash(q, q, q)
+    with pytest.raises(ValueError):
+        sd.qk_stats(q, q)

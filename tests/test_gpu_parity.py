@@ -1,0 +1,284 @@
+"""GPU parity: the CUDA kernels against the fp64 CPU oracle on the same seeded
+inputs (fp16 values widened exactly to fp64 on the oracle side).
+
+Gate (from the stated accuracy bar): over every compared output,
+max |O_gpu - O_ref| <= 2e-3 and ||O_gpu - O_ref||_F / ||O_ref||_F <= 1e-3.
+Also checked: A (fp32 scores) and L within 1e-4 absolute (fp32 sums of exact
+fp16 products), S within 1e-4 relative.  bf16 is reported against a looser
+bound (its 8-bit mantissa on P and O alone costs about 1.5e-3 relative).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import diffusion_unet_attention_b200 as sd  # noqa: E402
+
+DEV = torch.device("cuda:0")
+MAX_ABS, REL_FROB = 2e-3, 1e-3
+A_TOL, L_TOL, S_RTOL = 1e-4, 1e-4, 1e-4
+SENTINEL = 12345.0
+
+
+def f32(x):
+    return float(np.float32(x))
+
+
+def to_dev(*arrays):
+    return [torch.from_numpy(np.ascontiguousarray(a)).to(DEV) for a in arrays]
+
+
+def guarded(shape, dtype, pad=64):
+    """Output tensor with sentinel-filled margins before and after it."""
+    n = int(np.prod(shape))
+    buf = torch.full((n + 2 * pad,), SENTINEL, dtype=dtype, device=DEV)
+    return buf, buf[pad:pad + n].view(shape)
+
+
+def margins_intact(buf, pad=64):
+    h = buf[:pad].float().cpu().numpy()
+    t = buf[-pad:].float().cpu().numpy()
+    return bool(np.all(h == SENTINEL) and np.all(t == SENTINEL))
+
+
+def o_errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    diff = got - ref
+    return float(np.abs(diff).max()), float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+
+
+def assert_o(got, ref, what, max_abs=MAX_ABS, rel=REL_FROB):
+    ea, er = o_errors(got, ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert ea <= max_abs and er <= rel, f"{what}: max_abs {ea:.3e} rel_frob {er:.3e}"
+    return ea, er
+
+
+def run_paths(q, k, v, scale, rows=None, check_a=True):
+    """Runs both forms on the GPU; compares against the oracle on `rows`."""
+    B, H, N, d = q.shape
+    M = k.shape[2]
+    idx = np.arange(N) if rows is None else np.asarray(rows)
+    ref = oracle.attention(q[:, :, idx], k, v, scale, want_a=check_a)
+    tq, tk, tv = to_dev(q, k, v)
+    lda = (M + 3) // 4 * 4
+    obuf_f, o_f = guarded((B, H, N, d), tq.dtype)
+    obuf_p, o_p = guarded((B, H, N, d), tq.dtype)
+    abuf, a = guarded((B, H, N, lda), torch.float32)
+    lsbuf, ls = guarded((B, H, N, 2), torch.float32)
+    lsfbuf, lsf = guarded((B, H, N, 2), torch.float32)
+    sd.flash(tq, tk, tv, scale, out=o_f, out_ls=lsf)
+    sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls)
+    sd.softmax_av(a, ls, tv, scale, out=o_p)
+    torch.cuda.synchronize()
+    for name, buf in (("O flash", obuf_f), ("O partial", obuf_p), ("A", abuf), ("LS", lsbuf),
+                      ("LS flash", lsfbuf)):
+        assert margins_intact(buf), f"{name}: write outside the output"
+    res = {}
+    res["flash"] = assert_o(o_f[:, :, idx].float().cpu().numpy(), ref["O"], "flash")
+    res["partial"] = assert_o(o_p[:, :, idx].float().cpu().numpy(), ref["O"], "partially fused")
+    ls_h = ls[:, :, idx].cpu().numpy().astype(np.float64)
+    assert np.abs(ls_h[..., 0] - ref["L"]).max() <= L_TOL
+    assert np.abs(ls_h[..., 1] / ref["S"] - 1).max() <= S_RTOL
+    lsf_h = lsf[:, :, idx].cpu().numpy().astype(np.float64)
+    assert np.abs(lsf_h[..., 0] - ref["L"]).max() <= L_TOL
+    assert np.abs(lsf_h[..., 1] / ref["S"] - 1).max() <= S_RTOL
+    if check_a:
+        a_h = a[:, :, idx, :M].cpu().numpy().astype(np.float64)
+        assert np.abs(a_h - ref["A"]).max() <= A_TOL * (1 + np.abs(ref["A"]).max() / 8)
+    return res, (o_f, o_p, a, ls, lsf)
+
+
+# ---------------------------------------------------------------------------
+# the benchmark configurations
+# ---------------------------------------------------------------------------
+
+def test_tiny_config_fp32_inputs_rounded():
+    """Tiny config: fp32 N(0,1) inputs, rounded to fp16 (nearest even) on the
+    device; the gated oracle runs on the rounded values."""
+    shape = synth.CONFIGS[1]
+    q32, k32, v32 = synth.make_qkv(shape, 1, dtype=np.float32)
+    tq, tk, tv = (t.half() for t in to_dev(q32, k32, v32))
+    q, k, v = (t.cpu().numpy() for t in (tq, tk, tv))
+    assert np.array_equal(q, q32.astype(np.float16))
+    scale = f32(1 / math.sqrt(40))
+    run_paths(q, k, v, scale)
+    # reported, not gated: distance to the oracle on the unrounded fp32 inputs
+    raw = oracle.attention(q32, k32, v32, scale)
+    o = sd.flash(tq, tk, tv, scale).float().cpu().numpy()
+    ea, er = o_errors(o, raw["O"])
+    print(f"tiny config vs fp32-input oracle: max_abs {ea:.3e} rel_frob {er:.3e}")
+
+
+@pytest.mark.parametrize("cid", [3, 4, 5, 6])
+def test_config_full(cid):
+    shape = synth.CONFIGS[cid]
+    q, k, v = synth.make_qkv(shape, cid)
+    scale = f32(1 / math.sqrt(shape.d))
+    rows = None if shape.N <= 1024 else np.arange(0, shape.N, 3)
+    res, _ = run_paths(q, k, v, scale, rows=rows, check_a=shape.M <= 1024)
+    print(cid, res)
+
+
+def test_config_64x64_self_sampled():
+    """64x64-latent self-attention at full size (B=2, H=8, N=M=4096, d=40) in the
+    launch configuration the benchmark times; the oracle computes a sample of
+    query rows (every tile and the first and last rows of each)."""
+    shape = synth.CONFIGS[2]
+    q, k, v = synth.make_qkv(shape, 2)
+    scale = f32(1 / math.sqrt(40))
+    rows = np.unique(np.concatenate([np.arange(0, 4096, 61), np.arange(127, 4096, 128), [4095]]))
+    res, _ = run_paths(q, k, v, scale, rows=rows, check_a=True)
+    print(res)
+
+
+# ---------------------------------------------------------------------------
+# edge shapes: ragged tiles, single rows / keys, splits
+# ---------------------------------------------------------------------------
+EDGE = [
+    (1, 1, 1, 1, 40), (1, 1, 1, 77, 40), (1, 2, 129, 129, 40), (2, 1, 300, 77, 80),
+    (1, 1, 64, 64, 160), (1, 3, 257, 200, 160), (2, 2, 130, 1, 80), (1, 1, 128, 2053, 40),
+    (1, 1, 383, 1000, 80), (3, 1, 70, 65, 40), (1, 1, 2, 3, 160), (1, 2, 513, 511, 40),
+]
+
+
+@pytest.mark.parametrize("B,H,N,M,d", EDGE)
+def test_edge_shapes(B, H, N, M, d):
+    shape = synth.Shape("edge", B, H, N, M, d)
+    q, k, v = synth.make_qkv(shape, 40 + N % 7, call_id=M % 11)
+    run_paths(q, k, v, f32(1 / math.sqrt(d)))
+
+
+def test_peaked_scores_rescale():
+    """Q scaled x3 (scores with sigma ~ 3) and a late key that dominates: the
+    online max must grow across tiles and O must be rescaled."""
+    shape = synth.Shape("peaked", 1, 2, 256, 1024, 40)
+    q, k, v = synth.make_qkv(shape, 61)
+    q = (q.astype(np.float32) * 3).astype(np.float16)
+    k[:, :, 900] = (q[:, :, 0].astype(np.float32) * 2).astype(np.float16)
+    run_paths(q, k, v, f32(1 / math.sqrt(40)))
+
+
+# ---------------------------------------------------------------------------
+# invariants on the GPU outputs
+# ---------------------------------------------------------------------------
+
+def test_identical_keys_give_column_mean():
+    B, H, N, M, d = 1, 2, 200, 300, 40
+    q, _, v = synth.make_qkv(synth.Shape("t", B, H, N, M, d), 71)
+    k = np.repeat(synth.normal(72, (B, H, 1, d)), M, axis=2)
+    tq, tk, tv = to_dev(q, k, v)
+    mean = v.astype(np.float64).mean(axis=2, keepdims=True)
+    o = sd.flash(tq, tk, tv).float().cpu().numpy()
+    assert_o(o, np.broadcast_to(mean, o.shape), "flash identical keys")
+    o = sd.partially_fused(tq, tk, tv).float().cpu().numpy()
+    assert_o(o, np.broadcast_to(mean, o.shape), "partial identical keys")
+
+
+def test_one_hot_dominant_score():
+    B, H, N, M, d = 1, 1, 128, 256, 40
+    scale = f32(1 / math.sqrt(d))
+    beta = np.float16(30.0 / scale)
+    k = np.zeros((B, H, M, d), np.float16)
+    for j in range(d):
+        k[0, 0, j, j] = beta
+    perm = np.random.default_rng(5).permutation(N)
+    q = np.zeros((B, H, N, d), np.float16)
+    for i in range(N):
+        q[0, 0, i, perm[i] % d] = 1
+    v = synth.normal(73, (B, H, M, d))
+    tq, tk, tv = to_dev(q, k, v)
+    want = v[0, 0, perm % d].astype(np.float64)
+    for o in (sd.flash(tq, tk, tv, scale), sd.partially_fused(tq, tk, tv, scale)):
+        assert_o(o[0, 0].float().cpu().numpy(), want, "one-hot")
+
+
+def test_permutation_invariance():
+    shape = synth.Shape("t", 1, 2, 256, 384, 40)
+    q, k, v = synth.make_qkv(shape, 74)
+    perm = np.random.default_rng(9).permutation(384)
+    tq, tk, tv = to_dev(q, k, v)
+    tk2, tv2 = to_dev(k[:, :, perm], v[:, :, perm])
+    o1, ls1 = sd.flash(tq, tk, tv, return_ls=True)
+    o2, ls2 = sd.flash(tq, tk2, tv2, return_ls=True)
+    a1, l1 = sd.qk_stats(tq, tk)
+    a2, l2 = sd.qk_stats(tq, tk2)
+    # each score is the same fp32 dot product wherever its key sits
+    assert torch.equal(l1[..., 0], l2[..., 0])
+    assert torch.equal(ls1[..., 0], ls2[..., 0])
+    assert torch.equal(a1[..., :384][..., torch.from_numpy(perm).to(DEV)], a2[..., :384])
+    ea, er = o_errors(o2.float().cpu().numpy(), o1.float().cpu().numpy().astype(np.float64))
+    assert ea <= 1e-3 and er <= 1e-3
+
+
+def test_flash_and_partial_agree():
+    shape = synth.Shape("t", 2, 4, 512, 700, 80)
+    q, k, v = synth.make_qkv(shape, 75)
+    tq, tk, tv = to_dev(q, k, v)
+    of, lsf = sd.flash(tq, tk, tv, return_ls=True)
+    A, ls = sd.qk_stats(tq, tk)
+    op = sd.softmax_av(A, ls, tv)
+    assert torch.allclose(lsf[..., 0], ls[..., 0], atol=1e-5, rtol=0)
+    assert torch.allclose(lsf[..., 1], ls[..., 1], rtol=1e-4, atol=0)
+    ea, er = o_errors(of.float().cpu().numpy(), op.float().cpu().numpy().astype(np.float64))
+    assert ea <= 2e-3 and er <= 1e-3
+
+
+def test_repeated_calls_are_identical_and_workspace_resets():
+    """A split reduction (short rows, long keys) run twice: bitwise equal, and
+    the workspace's arrival counters are back at zero after each call."""
+    shape = synth.Shape("t", 1, 1, 256, 4096, 40)
+    q, k, v = synth.make_qkv(shape, 76)
+    tq, tk, tv = to_dev(q, k, v)
+    desc = sd.make_desc(1, 1, 256, 4096, 40, torch.float16, 1 / math.sqrt(40))
+    ws = sd.workspace(desc, DEV)
+    a1, l1 = sd.qk_stats(tq, tk, ws=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:8].sum()) == 0
+    a2, l2 = sd.qk_stats(tq, tk, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(l1, l2) and torch.equal(a1[..., :4096], a2[..., :4096])
+    ref = oracle.attention(q, k, v, f32(1 / math.sqrt(40)))
+    assert np.abs(l1.cpu().numpy()[..., 1] / ref["S"] - 1).max() <= S_RTOL
+
+
+def test_side_stream():
+    shape = synth.Shape("t", 2, 2, 300, 300, 40)
+    q, k, v = synth.make_qkv(shape, 77)
+    tq, tk, tv = to_dev(q, k, v)
+    ref = oracle.attention(q, k, v, f32(1 / math.sqrt(40)))
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        o = sd.flash(tq, tk, tv)
+        o2 = sd.partially_fused(tq, tk, tv)
+    s.synchronize()
+    assert_o(o.float().cpu().numpy(), ref["O"], "flash side stream")
+    assert_o(o2.float().cpu().numpy(), ref["O"], "partial side stream")
+
+
+def test_bf16_reported():
+    """bf16 is reported against a looser bound, not the fp16 gate."""
+    shape = synth.Shape("t", 1, 2, 256, 256, 40)
+    q, k, v = synth.make_qkv(shape, 78, dtype=np.float32)
+    tq, tk, tv = (t.bfloat16() for t in to_dev(q, k, v))
+    qb, kb, vb = (t.float().cpu().numpy() for t in (tq, tk, tv))
+    ref = oracle.attention(qb, kb, vb, f32(1 / math.sqrt(40)))
+    for name, o in (("flash", sd.flash(tq, tk, tv)), ("partial", sd.partially_fused(tq, tk, tv))):
+        ea, er = o_errors(o.float().cpu().numpy(), ref["O"])
+        print(f"bf16 {name}: max_abs {ea:.3e} rel_frob {er:.3e}")
+        assert ea <= 2e-2 and er <= 8e-3
+
+
+def test_no_device_error_recorded():
+    status, detail = sd.device_error()
+    assert status == "SDATTN_OK", (status, hex(detail))
