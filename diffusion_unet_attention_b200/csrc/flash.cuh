@@ -51,7 +51,7 @@ struct FlashCfg {
   static constexpr int K_BYTES = DSLABS * KV_SLAB;
   static constexpr int V_BYTES = DSLABS * KV_SLAB;
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int STAGES_FIT = (220 * 1024 - NQ * Q_TILE) / STAGE;
+  static constexpr int STAGES_FIT = (226 * 1024 - NQ * Q_TILE) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   static constexpr int QCOLS = SBUF * BN + PVN;     // tensor-memory columns per query tile
   static constexpr uint32_t TMEM_COLS = 512;
@@ -61,7 +61,9 @@ struct FlashCfg {
   static constexpr int NBAR = 2 + 3 * STAGES + NQ * SBUF + 2 * NQ + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
-  static_assert(STAGES >= 2, "need at least two key/value stages");
+  // With two S buffers the MMA issuer runs one tile further ahead, so the
+  // ring needs a third stage to keep loads overlapped with compute.
+  static_assert(STAGES >= 2 + (SBUF - 1), "key/value ring too shallow");
   static_assert(NQ * QCOLS <= 512, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
@@ -190,8 +192,15 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           const uint32_t kv = kv_base + j;
           const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
           const uint32_t t = t_base + j;
+          if (C::SBUF == 2 && j >= 2) {
+            // release tile j-2's stage before waiting for tile j's keys
+            for (int q = 0; q < NQ && live; ++q)
+              if (!issue_pv(q, j - 2)) live = false;
+            if (!live) break;
+            mma_commit(&kv_empty[(kv - 2) % C::STAGES]);
+          }
           for (int q = 0; q < NQ && live; ++q) {
-            if (j >= C::SBUF && !issue_pv(q, j - C::SBUF)) { live = false; break; }
+            if (C::SBUF == 1 && j >= 1 && !issue_pv(q, j - 1)) { live = false; break; }
             if (q == 0) {
               if (!mbar_wait(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
               tc_fence_after();
@@ -208,7 +217,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
             }
             mma_commit(&s_full[q * C::SBUF + (t % C::SBUF)]);
           }
-          if (live && j >= C::SBUF) mma_commit(&kv_empty[(kv - C::SBUF) % C::STAGES]);
+          if (C::SBUF == 1 && live && j >= 1) mma_commit(&kv_empty[(kv - 1) % C::STAGES]);
         }
         const int j0 = p.nkv > C::SBUF ? p.nkv - C::SBUF : 0;
         for (int jj = j0; jj < p.nkv && live; ++jj) {

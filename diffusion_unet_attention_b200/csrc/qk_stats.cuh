@@ -18,7 +18,8 @@
 //               through swizzled shared-memory staging and TMA stores.
 // When a row's columns are split over several units, each unit writes its
 // merged pair to the workspace and bumps an arrival counter; the unit that
-// arrives last merges all splits into LS and resets the counter (no spinning).
+// arrives last merges all splits into LS, then zeroes the partials it read and
+// the counter (no spinning), so a completed call leaves the workspace zero.
 #pragma once
 
 #include "sm100.cuh"
@@ -294,6 +295,8 @@ __global__ void __launch_bounds__(192, 1)
             const float2 q = __ldcg(pr + k);
             ms_merge(m, s, q.x, q.y);
           }
+          // leave the workspace all-zero for the next call, whatever its shape
+          for (int k = 0; k < p.nsplit; ++k) __stcg(const_cast<float2*>(pr) + k, make_float2(0.f, 0.f));
           if (row < p.N)
             *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(m, s);
           if (threadIdx.x == 64) p.tickets[tile] = 0u;

@@ -89,9 +89,10 @@ int64_t sdattn_a_ld(const sdattn_desc *desc);
 
 /* Bytes of workspace that sdattn_qk_stats and sdattn_softmax_av need for this
  * shape on the current device (split-reduction partials plus arrival
- * counters).  The same workspace serves both calls.  It must be zero-filled
- * once before its first use; every completed call leaves it ready for the next
- * (its counters back at zero).  Returns 0 for an invalid descriptor. */
+ * counters).  The same workspace serves both calls and any shape.  It must be
+ * zero-filled once before its first use; every completed call leaves all of
+ * it zero again.  After SDATTN_ERR_TIMEOUT it must be zero-filled anew.
+ * Returns 0 for an invalid descriptor. */
 size_t sdattn_workspace_bytes(const sdattn_desc *desc);
 
 /* Partially fused softmax, first kernel: the score matrix and its row
