@@ -1,0 +1,558 @@
+#!/usr/bin/env python
+"""Benchmark of the UNet attention hot path on B200.
+
+One step = the attention set of one 512x512 Stable Diffusion 1.4 UNet step:
+16 transformer blocks, each a self-attention (M = N = h*w) and a
+cross-attention (M = 77), B = 2 (classifier-free guidance pair), H = 8,
+d = 40 / 80 / 160, fp16 inputs.  Each call runs the form the paper's policy
+picks ("Speed Is All You Need", news summary, FlashAttention paragraph: the
+FlashAttention kernel for d = 40, the partially fused softmax elsewhere), so a
+step exercises every kernel: flash, qk_stats and softmax_av.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  `value` is whole-job TFLOP/s (algorithmic
+FLOPs 4*B*H*N*M*d summed over the set and over ranks, divided by the max-over-
+ranks device time of K steps).  Steps replay a CUDA graph of the set; two
+independent input sets (each larger than the 126 MB L2) alternate, so no step
+finds its inputs in L2.  Multi-GPU runs are independent replicas (the work
+needs no exchange); NCCL carries only the barrier and the max of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FLASH_SRC = ("diffusion_unet_attention_b200/csrc/flash.cuh", "diffusion_unet_attention_b200/csrc/sm100.cuh")
+PROFILE_MD = os.path.join(ROOT, "profiles", "flash_64x64_self_d40.md")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["sdattn", "reference"], default="sdattn")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--case", default=None,
+                    help="FORM:CONFIG, e.g. flash:2 -- run one form on one configuration (for profilers)")
+    ap.add_argument("--reps", type=int, default=3)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# workload
+# ----------------------------------------------------------------------------
+CALLS = synth.unet_step_set()
+STEP_FLOPS = sum(c.flops for c in CALLS)
+WORKLOAD = ("SD1.4 512x512 UNet step attention set: 16 transformer blocks x (self M=N=hw, cross M=77), "
+            "B=2, H=8, d=40/80/160, fp16 N(0,1); flash for d=40, partially fused softmax otherwise")
+
+
+def policy_form(call) -> str:
+    return "flash" if call.d == 40 else "partial"
+
+
+def is_dominant(call) -> bool:
+    return call.d == 40 and call.N == 4096 and call.M == 4096
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for rel in FLASH_SRC:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes of the flash kernel on the 64x64 self-attention,
+    from the committed ncu summary, if it was taken on the current source."""
+    try:
+        text = open(PROFILE_MD).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s*\(source\s+([0-9a-f]+)\)", text)
+    if not m or m.group(2) != source_digest():
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": statistics.median(power) if power else None}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+class StepSet:
+    """Device-resident inputs, outputs and scratch for one step set."""
+
+    def __init__(self, sd, torch, device, set_id: int):
+        self.sd, self.torch, self.device = sd, torch, device
+        self.inputs = []
+        for ci, call in enumerate(CALLS):
+            q, k, v = synth.make_qkv(call, synth.STEP_SET_ID + 10 * set_id, call_id=ci)
+            tq, tk, tv = (torch.from_numpy(x).to(device) for x in (q, k, v))
+            o = torch.empty_like(tq)
+            self.inputs.append((call, tq, tk, tv, o))
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for _, q, k, v, _ in self.inputs for t in (q, k, v))
+
+    def d2h_bytes(self):
+        return sum(o.numel() * o.element_size() for *_, o in self.inputs)
+
+
+class Scratch:
+    """A, LS and workspace shared by every partially fused call of a stream."""
+
+    def __init__(self, sd, torch, device, calls):
+        self.sd, self.torch = sd, torch
+        a_elems = max(c.B * c.H * c.N * ((c.M + 3) // 4 * 4) for c in calls)
+        ls_elems = max(c.B * c.H * c.N * 2 for c in calls)
+        self.a = torch.empty(a_elems, dtype=torch.float32, device=device)
+        self.ls = torch.empty(ls_elems, dtype=torch.float32, device=device)
+        ws = max(sd.workspace_bytes(sd.make_desc(c.B, c.H, c.N, c.M, c.d, torch.float16, 1.0)) for c in calls)
+        self.ws = torch.zeros(max(ws, 256), dtype=torch.uint8, device=device)
+
+    def run(self, call, q, k, v, o, form):
+        sd = self.sd
+        scale = 1.0 / math.sqrt(call.d)
+        if form == "flash":
+            sd.flash(q, k, v, scale, out=o)
+            return 1
+        lda = (call.M + 3) // 4 * 4
+        a = self.a[:call.B * call.H * call.N * lda].view(call.B, call.H, call.N, lda)
+        ls = self.ls[:call.B * call.H * call.N * 2].view(call.B, call.H, call.N, 2)
+        sd.qk_stats(q, k, scale, out_a=a, out_ls=ls, ws=self.ws)
+        sd.softmax_av(a, ls, v, scale, out=o)
+        return 2
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import diffusion_unet_attention_b200 as sd
+
+    sd.load_library()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        from datetime import timedelta
+        dist_mod.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+        dist = dist_mod
+
+    stream = torch.cuda.Stream(device)
+    sets = [StepSet(sd, torch, device, s) for s in range(2)]
+    scratch = Scratch(sd, torch, device, CALLS)
+    dom_calls = [i for i, c in enumerate(CALLS) if is_dominant(c)]
+    rest_calls = [i for i, c in enumerate(CALLS) if not is_dominant(c)]
+
+    def issue(stepset, idxs, form_of):
+        n = 0
+        for i in idxs:
+            call, q, k, v, o = stepset.inputs[i]
+            n += scratch.run(call, q, k, v, o, form_of(call))
+        return n
+
+    # ---- capture: per input set, the dominant segment and the rest ----------
+    launches_per_step = 0
+    graphs = []
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for s in sets:               # eager warm-up of every kernel variant before capture
+            issue(s, range(len(CALLS)), policy_form)
+        stream.synchronize()
+        for s in sets:
+            g_dom, g_rest = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_dom, stream=stream):
+                n1 = issue(s, dom_calls, policy_form)
+            with torch.cuda.graph(g_rest, stream=stream):
+                n2 = issue(s, rest_calls, policy_form)
+            graphs.append((g_dom, g_rest))
+            launches_per_step = n1 + n2
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            g_dom, g_rest = graphs[i % 2]
+            g_dom.replay()
+            g_rest.replay()
+    ev_dom = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(visible.split(",")[local_rank].strip() if visible else str(local_rank))
+    barrier()
+    clocks.start()
+    time.sleep(0.3)
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(K):
+            g_dom, g_rest = graphs[i % 2]
+            ev_dom[i][0].record(stream)
+            g_dom.replay()
+            ev_dom[i][1].record(stream)
+            g_rest.replay()
+        t1.record(stream)
+    stream.synchronize()
+    wall = time.time() - wall0
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    dom_ms = sum(a.elapsed_time(b) for a, b in ev_dom) / (K * len(dom_calls))
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / K
+    value = world * STEP_FLOPS * K / (elapsed_ms * 1e-3) / 1e12
+
+    extra = {}
+    e2e = None
+    if rank == 0:
+        extra = side_measurements(torch, sd, stream, sets, scratch, issue, K=min(K, 50))
+        e2e = end_to_end(torch, sd, stream, sets[0], scratch, steps=min(K, 10))
+
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    dom_flops = synth.CONFIGS[2].flops
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    traffic = profiled_traffic()
+    line = {
+        "metric": "attention us & TFLOP/s per UNet-step set (1xB200); % of tensor / HBM roofline",
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic N(0,1), seeded SplitMix64/Box-Muller, fp16",
+        "config": {"workload": WORKLOAD, "calls_per_step": len(CALLS), "flops_per_step": STEP_FLOPS,
+                   "accumulate": "f32", "l2": "two input sets of %.0f MB alternate (each > 126 MB L2)"
+                   % (sets[0].h2d_bytes() / 1e6), "timing": "CUDA graph replay per step, CUDA events",
+                   "parallelism": f"replicas x{world}"},
+        "gpu_launches": launches_per_step * K,
+        "roofline": {"bound": "tensor", "kernel": "flash_kernel<40,2,128> on 64x64 self-attention",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 dense burst (fp16 dense has the same nominal rate)",
+                     "flops_per_launch": dom_flops, "avg_launch_us": round(dom_ms * 1e3, 3)},
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
+                   "samples": clk["samples"], "power_w_median": clk.get("power_w_median")},
+        "wall_s_timed": round(wall, 3),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    line.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def side_measurements(torch, sd, stream, sets, scratch, issue, K):
+    """Per-form step-set times and the two headline kernels on the 64x64
+    self-attention, each timed with CUDA events (graph replays)."""
+    out = {}
+
+    def time_graph(build, reps, per_rep_div=1):
+        gs = []
+        with torch.cuda.stream(stream):
+            for s in sets:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    build(s)
+                gs.append(g)
+            for i in range(3):
+                gs[i % 2].replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(reps):
+                gs[i % 2].replay()
+            b.record(stream)
+        stream.synchronize()
+        del gs
+        return a.elapsed_time(b) / reps / per_rep_div
+
+    forms = {}
+    for name, fn in (("flash_all", lambda c: "flash"), ("partial_all", lambda c: "partial"),
+                     ("policy", policy_form)):
+        ms = time_graph(lambda s, fn=fn: issue(s, range(len(CALLS)), fn), K)
+        forms[name] = {"ms_per_step": round(ms, 5), "tflops": round(STEP_FLOPS / (ms * 1e-3) / 1e12, 2)}
+    out["forms"] = forms
+
+    # headline kernels on the 64x64 self-attention (5 distinct calls per replay)
+    dom = [i for i, c in enumerate(CALLS) if is_dominant(c)]
+    c2 = synth.CONFIGS[2]
+    peaks, _ = measured_peaks()
+    f_ms = time_graph(lambda s: issue(s, dom, lambda c: "flash"), K, len(dom))
+    p_ms = time_graph(lambda s: issue(s, dom, lambda c: "partial"), max(K // 4, 5), len(dom))
+    pf_bytes = 2 * c2.a_bytes() + 4 * c2.B * c2.H * c2.N * c2.d * 2 + c2.B * c2.H * c2.N * 8
+    out["kernels_64x64_self"] = {
+        "flash": {"us": round(f_ms * 1e3, 2), "tflops": round(c2.flops / (f_ms * 1e-3) / 1e12, 1),
+                  "frac_measured_tensor_peak": round(c2.flops / (f_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                  "frac_2250_tflops": round(c2.flops / (f_ms * 1e-3) / 2.25e15, 4)},
+        "partially_fused": {"us": round(p_ms * 1e3, 2), "gbs": round(pf_bytes / (p_ms * 1e-3) / 1e9, 1),
+                            "algorithmic_bytes": pf_bytes,
+                            "frac_measured_hbm": round(pf_bytes / (p_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+    }
+    return out
+
+
+def end_to_end(torch, sd, stream, stepset, scratch, steps):
+    """The same metric through the public API with host buffers: every step
+    copies its inputs from pinned host memory, runs the set, reads O back."""
+    host_in = []
+    for call, q, k, v, o in stepset.inputs:
+        host_in.append(tuple(t.cpu().pin_memory() for t in (q, k, v)))
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for *_, o in stepset.inputs]
+    dev = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(o))
+           for _, q, k, v, o in stepset.inputs]
+    h2d = sum(t.numel() * t.element_size() for tr in host_in for t in tr)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def one_step():
+        for (call, *_), (hq, hk, hv), (dq, dk, dv, do), ho in zip(stepset.inputs, host_in, dev, host_out):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            scratch.run(call, dq, dk, dv, do, policy_form(call))
+            ho.copy_(do, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        one_step()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            one_step()
+        b.record(stream)
+    stream.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return {"value": round(STEP_FLOPS / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "path": "public Python API (ctypes -> C ABI), pinned host buffers, eager launches"}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(row_stride: int, seed_offset: int = 0):
+    """Runs the fp64 oracle on every `row_stride`-th query row of every call of
+    the step set; returns (algorithmic FLOPs done, seconds, threads)."""
+    import oracle
+    lib = oracle.load()
+    flops, secs = 0, 0.0
+    for ci, call in enumerate(CALLS):
+        q, k, v = synth.make_qkv(call, synth.STEP_SET_ID + seed_offset, call_id=ci)
+        qs = np.ascontiguousarray(q[:, :, ::row_stride])
+        t = time.perf_counter()
+        oracle.attention(qs, k, v, 1.0 / math.sqrt(call.d), lib=lib)
+        secs += time.perf_counter() - t
+        flops += 4 * call.B * call.H * qs.shape[2] * call.M * call.d
+    return flops, secs, oracle.max_threads()
+
+
+def choose_stride(budget_s: float) -> int:
+    """Row stride whose oracle sample takes about budget_s seconds."""
+    f, s, _ = oracle_sample(4096)
+    rate = f / max(s, 1e-6)
+    want = budget_s * rate
+    return max(1, int(STEP_FLOPS / max(want, 1.0)))
+
+
+def cpu_baseline(seconds: float):
+    stride = choose_stride(seconds)
+    f, s, thr = oracle_sample(stride)
+    return {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+            "sample": f"every {stride}-th query row of all 32 calls of the step set "
+                      f"({f / 1e9:.2f} GFLOP of the {STEP_FLOPS / 1e9:.1f} GFLOP step), fp64 C + OpenMP",
+            "seconds": round(s, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    K, W = args.steps, args.warmup
+    budget = 90.0 / max(K + W, 1)          # whole run about a minute and a half
+    stride = choose_stride(budget)
+    for _ in range(W):
+        oracle_sample(stride)
+    tot_f, tot_s, thr = 0, 0.0, 1
+    for _ in range(K):
+        f, s, thr = oracle_sample(stride)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    line = {"metric": "attention us & TFLOP/s per UNet-step set (1xB200); % of tensor / HBM roofline",
+            "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": round(STEP_FLOPS / (value * 1e12) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD}, "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                             "sample": f"every {stride}-th query row of all 32 calls per step"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_case(args):
+    """One form on one configuration, `reps` launches after one warm-up, each
+    timed with CUDA events; used as the target of profiler captures."""
+    import torch
+    import diffusion_unet_attention_b200 as sd
+    form, cid = args.case.split(":")
+    call = synth.CONFIGS[int(cid)]
+    device = torch.device("cuda", 0)
+    q, k, v = synth.make_qkv(call, int(cid))
+    tq, tk, tv = (torch.from_numpy(x).to(device) for x in (q, k, v))
+    o = torch.empty_like(tq)
+    scratch = Scratch(sd, torch, device, [call])
+    scale = 1.0 / math.sqrt(call.d)
+    lda = (call.M + 3) // 4 * 4
+    a = scratch.a[:call.B * call.H * call.N * lda].view(call.B, call.H, call.N, lda)
+    ls = scratch.ls[:call.B * call.H * call.N * 2].view(call.B, call.H, call.N, 2)
+
+    def once():
+        if form == "flash":
+            sd.flash(tq, tk, tv, scale, out=o)
+        elif form == "qk_stats":
+            sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
+        elif form == "softmax_av":
+            sd.softmax_av(a, ls, tv, scale, out=o)
+        else:
+            scratch.run(call, tq, tk, tv, o, "partial")
+
+    if form == "softmax_av":
+        sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
+    once()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        once()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    status = sd.device_error()
+    print(json.dumps({"case": args.case, "shape": call.__dict__, "us": [round(t, 2) for t in times],
+                      "device_error": status[0]}), flush=True)
+    if status[0] != "SDATTN_OK":
+        sys.exit(1)
+
+
+def main():
+    args = parse_args()
+    if args.case:
+        run_case(args)
+        return
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

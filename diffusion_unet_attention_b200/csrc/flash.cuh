@@ -69,7 +69,7 @@ struct FlashCfg {
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
 };
 
-template <int D, int NQ, int BN, bool BF16>
+template <int D, int NQ, int BN, bool BF16, int NPOLY>
 __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     flash_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
+    if constexpr (NQ == 2) regs_dec<120>();
     if (lane == 0) {
       uint32_t kvc = 0, nq = 0;
       bool live = true;
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
+    if constexpr (NQ == 2) regs_dec<120>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16(128, BN, BF16, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(128, C::PVN, BF16, false, true);
@@ -235,20 +237,37 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     }
   } else if (warp >= 4) {
     // ---------------------------- softmax, tile q -----------------------------
+    if constexpr (NQ == 2) regs_inc<192>();
     const int q = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t o_tmem = tmem + q * C::QCOLS + C::SBUF * BN + lane_off;
     const float c = p.c;
-    uint32_t t = 0;       // tiles seen by this query-tile slot (all units)
+    // V's padding column D is set to 1 in every tile, so column D of O
+    // accumulates the row sum of P in fp32 on the tensor core.
+    constexpr int TAIL = D - 64 * (C::DSLABS - 1);           // columns of V's last slab
+    const uint32_t one16 = BF16 ? 0x3F80u : 0x3C00u;
+    uint32_t t = 0;        // tiles seen by this query-tile slot (all units)
+    uint32_t kvt = 0;      // key tiles seen (stage index)
     bool live = true;
     for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
       const int bh = u / p.tph, qg = u % p.tph;
       const int row = (qg * NQ + q) * 128 + r;
-      float m_used = -INFINITY, l = 0.f, rawmax = -INFINITY;
-      for (int j = 0; j < p.nkv; ++j, ++t) {
+      float m_used = -INFINITY, rawmax = -INFINITY;
+      for (int j = 0; j < p.nkv; ++j, ++t, ++kvt) {
         const uint32_t slot = t % C::SBUF, n = t / C::SBUF;
+        if (q == 0) {
+          // ones column of this tile's V rows (after the tile has landed)
+          const uint32_t st = kvt % C::STAGES, ns = kvt / C::STAGES;
+          live = __all_sync(0xffffffffu, mbar_wait(&v_full[st], ns & 1, kSiteVFull, abort_flag));
+          if (!live) break;
+          if (r < BN) {
+            uint8_t* vrow = sKV + st * C::STAGE + C::K_BYTES + (C::DSLABS - 1) * C::KV_SLAB + r * 128;
+            *reinterpret_cast<uint4*>(vrow + (((TAIL / 8) ^ (r & 7)) << 4)) = make_uint4(one16, 0u, 0u, 0u);
+            fence_proxy_async_smem();
+          }
+        }
         live = __all_sync(0xffffffffu, mbar_wait(&s_full[q * C::SBUF + slot], n & 1, kSiteSFull, abort_flag));
         if (!live) break;
         tc_fence_after();
@@ -264,26 +283,44 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           for (int k = 0; k < BN; ++k)
             if (k >= valid) v[k] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(v[0]);
+        // row max: eight independent three-input chains, then a small tree
+        float acc[8];
 #pragma unroll
-        for (int k = 1; k < BN; ++k) mx = fmaxf(mx, __uint_as_float(v[k]));
+        for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(v[i]);
+        int k0 = 8;
+#pragma unroll
+        for (; k0 + 16 <= BN; k0 += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[i] = fmax3(acc[i], __uint_as_float(v[k0 + i]), __uint_as_float(v[k0 + 8 + i]));
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (k0 + i < BN) acc[i] = fmaxf(acc[i], __uint_as_float(v[k0 + i]));
+        const float mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7])));
         rawmax = fmaxf(rawmax, mx);
         const float mt = mx * c;
         float alpha = 1.f;
         bool rescale = false;
         if (mt > m_used + 8.f) {
           alpha = ex2_approx(m_used - mt);
-          l *= alpha;
           m_used = mt;
           rescale = (j > 0);
         }
-        const float nm = -m_used;
+        // p = 2^(s*c - m): NPOLY of every 8 pairs on the FMA pipe, the rest on MUFU
+        const uint64_t c2 = f2_pack(c, c);
+        const uint64_t nm2 = f2_pack(-m_used, -m_used);
         uint32_t pk[BN / 2];
 #pragma unroll
         for (int k = 0; k < BN / 2; ++k) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(v[2 * k]), c, nm));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(v[2 * k + 1]), c, nm));
-          l += e0 + e1;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), c2, nm2);
+          float x0, x1, e0, e1;
+          f2_unpack(x2, x0, x1);
+          if ((k & 7) < NPOLY) {
+            exp2_poly2(x0, x1, e0, e1);
+          } else {
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+          }
           pk[k] = pack2<BF16>(e0, e1);
         }
 #pragma unroll
@@ -313,10 +350,18 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[q]);
       }
       if (!live) break;
-      // ---- epilogue: O / l ----
+      // ---- epilogue: O / l, with l = column D of O ----
       live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
       if (!live) break;
       tc_fence_after();
+      float l;
+      {
+        uint32_t o[8];
+        tmem_ld_x8(o_tmem + D, o);
+        tmem_wait_ld();
+        reg_fence<8>(o);
+        l = __uint_as_float(o[0]);
+      }
       const float inv = 1.f / l;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row) * D * 2;
 #pragma unroll
@@ -339,6 +384,9 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       }
       tc_fence_before();
     }
+  } else {
+    // idle warps of the first warp group
+    if constexpr (NQ == 2) regs_dec<120>();
   }
 
   tc_fence_before();

@@ -227,13 +227,13 @@ sdattn_status launch_av(const sdattn_desc* d, const float* A, const float* LS, c
   return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
-template <int D, int NQ, int BN, bool BF16>
+template <int D, int NQ, int BN, bool BF16, int NPOLY = 3>
 sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
                            cudaStream_t stream) {
   using C = FlashCfg<D, NQ, BN>;
   const int dev = current_device();
   if (dev < 0) return SDATTN_ERR_CUDA;
-  auto kern = sdattn::flash_kernel<D, NQ, BN, BF16>;
+  auto kern = sdattn::flash_kernel<D, NQ, BN, BF16, NPOLY>;
   static std::atomic<uint64_t> smem_done{0};
   if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
 

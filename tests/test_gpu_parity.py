@@ -4,8 +4,12 @@ inputs (fp16 values widened exactly to fp64 on the oracle side).
 Gate (from the stated accuracy bar): over every compared output,
 max |O_gpu - O_ref| <= 2e-3 and ||O_gpu - O_ref||_F / ||O_ref||_F <= 1e-3.
 Also checked: A (fp32 scores) and L within 1e-4 absolute (fp32 sums of exact
-fp16 products), S within 1e-4 relative.  bf16 is reported against a looser
-bound (its 8-bit mantissa on P and O alone costs about 1.5e-3 relative).
+fp16 products); S within 1e-4 relative from qk_stats (fp32 exponentials).
+The flash kernel's S is the tensor-core sum of the 16-bit P it multiplies with
+V (a ones column in V's padding), so each term carries one fp16 rounding:
+|sum fl(p) - sum p| <= 2^-11 sum p for p >= 0, plus the 7.5e-5 bound of its
+polynomial exponential, hence 6e-4 relative.  bf16 is reported against a
+looser bound (its 8-bit mantissa on P and O alone costs about 1.5e-3 relative).
 """
 import math
 
@@ -25,7 +29,7 @@ import diffusion_unet_attention_b200 as sd  # noqa: E402
 
 DEV = torch.device("cuda:0")
 MAX_ABS, REL_FROB = 2e-3, 1e-3
-A_TOL, L_TOL, S_RTOL = 1e-4, 1e-4, 1e-4
+A_TOL, L_TOL, S_RTOL, S_RTOL_FLASH = 1e-4, 1e-4, 1e-4, 6e-4
 SENTINEL = 12345.0
 
 
@@ -92,7 +96,7 @@ def run_paths(q, k, v, scale, rows=None, check_a=True):
     assert np.abs(ls_h[..., 1] / ref["S"] - 1).max() <= S_RTOL
     lsf_h = lsf[:, :, idx].cpu().numpy().astype(np.float64)
     assert np.abs(lsf_h[..., 0] - ref["L"]).max() <= L_TOL
-    assert np.abs(lsf_h[..., 1] / ref["S"] - 1).max() <= S_RTOL
+    assert np.abs(lsf_h[..., 1] / ref["S"] - 1).max() <= S_RTOL_FLASH
     if check_a:
         a_h = a[:, :, idx, :M].cpu().numpy().astype(np.float64)
         assert np.abs(a_h - ref["A"]).max() <= A_TOL * (1 + np.abs(ref["A"]).max() / 8)
@@ -229,7 +233,7 @@ def test_flash_and_partial_agree():
     A, ls = sd.qk_stats(tq, tk)
     op = sd.softmax_av(A, ls, tv)
     assert torch.allclose(lsf[..., 0], ls[..., 0], atol=1e-5, rtol=0)
-    assert torch.allclose(lsf[..., 1], ls[..., 1], rtol=1e-4, atol=0)
+    assert torch.allclose(lsf[..., 1], ls[..., 1], rtol=S_RTOL_FLASH + S_RTOL, atol=0)
     ea, er = o_errors(of.float().cpu().numpy(), op.float().cpu().numpy().astype(np.float64))
     assert ea <= 2e-3 and er <= 1e-3
 
