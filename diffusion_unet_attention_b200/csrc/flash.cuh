@@ -17,12 +17,17 @@
 //   warps 4+4q..7+4q  softmax for query tile q, one row per thread: row max,
 //                     p = 2^(s*scale*log2e - m), row sum, P packed to 16 bits,
 //                     and the rescale of O when the running max grows.
-// With NQ = 2 the two tiles ping-pong: while one tile's softmax runs, the
-// tensor core computes the other's scores.  With NQ = 1 the S buffer is
-// doubled instead, so the next tile's scores are ready when the softmax is.
+// S, P and O have separate tensor-memory buffers per query tile.  The softmax
+// releases S as soon as it has loaded it into registers, so the tensor core
+// computes the next tile's scores while this tile's exponentials run; P is
+// released when P V completes.  With NQ = 2 two query tiles share the key
+// and value stages and their softmax phases overlap on the SM.
 // The running max is only raised when a tile's max exceeds it by more than
 // 2^8 (in the base-2 exponent), so O is rescaled rarely; p stays below 256,
 // which 16-bit P and the fp32 accumulators absorb exactly as the true max would.
+// The row sum l comes from the tensor core: V's padding column D holds 1 in
+// every stage (written once; the V tile loads never cover it), so column D of
+// O accumulates sum_j p_j from the same 16-bit P that multiplies V.
 #pragma once
 
 #include "sm100.cuh"
@@ -44,35 +49,40 @@ template <int D, int NQ, int BN>
 struct FlashCfg {
   static constexpr int DSLABS = (D + 63) / 64;
   static constexpr int KSTEPS = (D + 15) / 16;
-  static constexpr int PVN = DSLABS * 64;
-  static constexpr int SBUF = NQ == 1 ? 2 : 1;     // S/P buffers per query tile
+  static constexpr int PVN = DSLABS * 64;          // P V width: D padded to 64, column D = row sum
+  static constexpr int TAIL = D - 64 * (DSLABS - 1);  // V columns loaded into its last slab
   static constexpr int Q_TILE = DSLABS * 128 * 128;
   static constexpr int KV_SLAB = BN * 128;
   static constexpr int K_BYTES = DSLABS * KV_SLAB;
   static constexpr int V_BYTES = DSLABS * KV_SLAB;
+  static constexpr int V_TX = (DSLABS - 1) * KV_SLAB + TAIL * 2 * BN;   // bytes the V loads deliver
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int STAGES_FIT = (226 * 1024 - NQ * Q_TILE) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
-  static constexpr int QCOLS = SBUF * BN + PVN;     // tensor-memory columns per query tile
-  static constexpr uint32_t TMEM_COLS = 512;
+  // tensor memory per query tile: S (BN fp32), P (BN/2 columns of 16-bit pairs), O (PVN fp32)
+  static constexpr uint32_t TM_S = 0;
+  static constexpr uint32_t TM_P = BN;
+  static constexpr uint32_t TM_O = BN + BN / 2;
+  static constexpr int QCOLS = BN + BN / 2 + PVN;
+  static constexpr uint32_t TMEM_COLS = NQ * QCOLS <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = NQ * Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
-  static constexpr int NBAR = 2 + 3 * STAGES + NQ * SBUF + 2 * NQ + 1;
+  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
-  // With two S buffers the MMA issuer runs one tile further ahead, so the
-  // ring needs a third stage to keep loads overlapped with compute.
-  static_assert(STAGES >= 2 + (SBUF - 1), "key/value ring too shallow");
+  static_assert(STAGES >= 2, "key/value ring too shallow");
   static_assert(NQ * QCOLS <= 512, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
+  static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
 };
 
 template <int D, int NQ, int BN, bool BF16, int NPOLY>
 __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     flash_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const FlashParams p) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmVt,
+                 const FlashParams p) {
   using C = FlashCfg<D, NQ, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,10 +94,12 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   uint64_t* k_full = bars + 2;
   uint64_t* v_full = k_full + C::STAGES;
   uint64_t* kv_empty = v_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;          // [NQ][SBUF]
-  uint64_t* p_full = s_full + NQ * C::SBUF;         // [NQ]
-  uint64_t* pv_done = p_full + NQ;                  // [NQ]
-  uint64_t* drain_bar = pv_done + NQ;
+  // The NQ query tiles advance in lockstep, so each handshake has one barrier:
+  uint64_t* s_full = kv_empty + C::STAGES;   // MMA -> softmax: S of every query tile ready
+  uint64_t* s_free = s_full + 1;             // softmax -> MMA: S loaded, buffers free
+  uint64_t* p_full = s_free + 1;             // softmax -> MMA: P written (O rescaled)
+  uint64_t* pv_done = p_full + 1;            // MMA -> softmax: P V done, P buffers free
+  uint64_t* drain_bar = pv_done + 1;
   uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
@@ -102,19 +114,33 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < NQ * C::SBUF; ++i) mbar_init(&s_full[i], 1);
-    for (int i = 0; i < NQ; ++i) {
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4 * NQ);
+    mbar_init(p_full, 4 * NQ);
+    mbar_init(pv_done, 1);
     mbar_init(drain_bar, 1);
     misc[1] = 0;
     fence_mbar_init();
+  }
+  // V's last slab: the loads cover its first TAIL columns; column D (chunk
+  // TAIL/8 of each 128-byte row, element 0) holds 1 and the rest 0, for good.
+  {
+    const uint32_t one16 = BF16 ? 0x3F80u : 0x3C00u;
+    for (int i = threadIdx.x; i < C::STAGES * BN; i += blockDim.x) {
+      const int st = i / BN, r = i % BN;
+      uint8_t* row = sKV + st * C::STAGE + C::K_BYTES + (C::DSLABS - 1) * C::KV_SLAB + r * 128;
+#pragma unroll
+      for (int ch = C::TAIL / 8; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) =
+            make_uint4(ch == C::TAIL / 8 ? one16 : 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
   }
   if (threadIdx.x == 32) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmVt);
   }
   if (warp == 1) {
     tmem_alloc(&misc[0], C::TMEM_COLS);
@@ -146,8 +172,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           uint8_t* sV = sK + C::K_BYTES;
           mbar_arrive_expect_tx(&k_full[st], C::K_BYTES);
           for (int s = 0; s < C::DSLABS; ++s) tma_load_3d(sK + s * C::KV_SLAB, &tmK, 64 * s, j * BN, bh, &k_full[st]);
-          mbar_arrive_expect_tx(&v_full[st], C::V_BYTES);
-          for (int s = 0; s < C::DSLABS; ++s) tma_load_3d(sV + s * C::KV_SLAB, &tmV, 64 * s, j * BN, bh, &v_full[st]);
+          mbar_arrive_expect_tx(&v_full[st], C::V_TX);
+          for (int s = 0; s + 1 < C::DSLABS; ++s)
+            tma_load_3d(sV + s * C::KV_SLAB, &tmV, 64 * s, j * BN, bh, &v_full[st]);
+          tma_load_3d(sV + (C::DSLABS - 1) * C::KV_SLAB, &tmVt, 64 * (C::DSLABS - 1), j * BN, bh, &v_full[st]);
         }
       }
       volatile uint32_t never = 0;
@@ -160,81 +188,61 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
+    // The whole warp runs the loop; one elected lane issues.  Per key tile j:
+    // S_j for every query tile (once the softmax has loaded S_{j-1}), then
+    // P V for tile j-1 (once P_{j-1} is written).
     if constexpr (NQ == 2) regs_dec<120>();
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f16(128, BN, BF16, false, false);
-      constexpr uint32_t idesc_pv = idesc_f16(128, C::PVN, BF16, false, true);
-      const uint32_t q_base = smem_u32(sQ), kv_base_addr = smem_u32(sKV);
-      uint32_t t_base = 0, kv_base = 0, ui = 0;
-      bool live = true;
-
-      auto issue_pv = [&](int q, int jj) -> bool {
-        const uint32_t kv = kv_base + jj;
-        const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
-        const uint32_t t = t_base + jj;
-        if (q == 0 && !mbar_wait(&v_full[st], n & 1, kSiteVFull, abort_flag)) return false;
-        if (!mbar_wait(&p_full[q], t & 1, kSitePFull, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + q * C::QCOLS + (t % C::SBUF) * BN;
-        const uint32_t o_tmem = tmem + q * C::QCOLS + C::SBUF * BN;
-        const uint32_t v_addr = kv_base_addr + st * C::STAGE + C::K_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, C::KV_SLAB, 1024);
-          mma_ts(o_tmem, p_tmem + kk * 8, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&pv_done[q]);
-        return true;
-      };
-
-      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
-        if (!mbar_wait(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
-        tc_fence_after();
-        for (int j = 0; j < p.nkv && live; ++j) {
-          const uint32_t kv = kv_base + j;
+    constexpr uint32_t idesc_s = idesc_f16(128, BN, BF16, false, false);
+    constexpr uint32_t idesc_pv = idesc_f16(128, C::PVN, BF16, false, true);
+    // descriptors of the first Q slab and of stage 0's K and V; others by address offset
+    const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);
+    const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV) + C::K_BYTES, C::KV_SLAB, 1024);
+    uint32_t t_base = 0, kv_base = 0, ui = 0;
+    bool live = true;
+    for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
+      if (!mbar_wait_warp(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
+      for (int j = 0; j <= p.nkv; ++j) {
+        if (j < p.nkv) {
+          const uint32_t kv = kv_base + j, t = t_base + j;
           const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
-          const uint32_t t = t_base + j;
-          if (C::SBUF == 2 && j >= 2) {
-            // release tile j-2's stage before waiting for tile j's keys
-            for (int q = 0; q < NQ && live; ++q)
-              if (!issue_pv(q, j - 2)) live = false;
-            if (!live) break;
-            mma_commit(&kv_empty[(kv - 2) % C::STAGES]);
-          }
-          for (int q = 0; q < NQ && live; ++q) {
-            if (C::SBUF == 1 && j >= 1 && !issue_pv(q, j - 1)) { live = false; break; }
-            if (q == 0) {
-              if (!mbar_wait(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
-              tc_fence_after();
-            }
-            const uint32_t s_tmem = tmem + q * C::QCOLS + (t % C::SBUF) * BN;
-            const uint32_t k_addr = kv_base_addr + st * C::STAGE;
+          if (!mbar_wait_warp(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
+          if (t >= 1 && !mbar_wait_warp(s_free, (t - 1) & 1, kSiteSFull, abort_flag)) { live = false; break; }
+          tc_fence_after();
+          const uint64_t kd = k_desc0 + ((st * C::STAGE) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t koff = (kk >> 2) * C::KV_SLAB + (kk & 3) * 32;
-              const uint64_t ad = sdesc_sw128(q_base + q * C::Q_TILE + off, 16, 1024);
-              const uint64_t bd = sdesc_sw128(k_addr + koff, 16, 1024);
-              mma_ss(s_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&s_full[q * C::SBUF + (t % C::SBUF)]);
-          }
-          if (C::SBUF == 1 && live && j >= 1) mma_commit(&kv_empty[(kv - 1) % C::STAGES]);
+          for (int q = 0; q < NQ; ++q)
+#pragma unroll
+            for (int kk = 0; kk < C::KSTEPS; ++kk)
+              mma_ss(tmem + q * C::QCOLS + C::TM_S,
+                     q_desc0 + ((q * C::Q_TILE + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                     kd + (((kk >> 2) * C::KV_SLAB + (kk & 3) * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
+          mma_commit(s_full);
         }
-        const int j0 = p.nkv > C::SBUF ? p.nkv - C::SBUF : 0;
-        for (int jj = j0; jj < p.nkv && live; ++jj) {
-          for (int q = 0; q < NQ && live; ++q)
-            if (!issue_pv(q, jj)) live = false;
-          if (live) mma_commit(&kv_empty[(kv_base + jj) % C::STAGES]);
+        if (j >= 1) {
+          const uint32_t kv = kv_base + j - 1, t = t_base + j - 1;
+          const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
+          if (!mbar_wait_warp(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait_warp(p_full, t & 1, kSitePFull, abort_flag)) { live = false; break; }
+          tc_fence_after();
+          const uint64_t vd = v_desc0 + ((st * C::STAGE) >> 4);
+#pragma unroll
+          for (int q = 0; q < NQ; ++q)
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ts(tmem + q * C::QCOLS + C::TM_O, tmem + q * C::QCOLS + C::TM_P + kk * 8,
+                     vd + ((kk * 2048) >> 4), idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+          mma_commit(pv_done);
+          mma_commit(&kv_empty[st]);
         }
-        if (live) mma_commit(q_empty);
-        t_base += p.nkv;
-        kv_base += p.nkv;
       }
-      volatile uint32_t never = 0;
-      mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kSitePvDone, &never);
+      if (live) mma_commit(q_empty);
+      t_base += p.nkv;
+      kv_base += p.nkv;
     }
+    volatile uint32_t never = 0;
+    mma_commit(drain_bar);
+    mbar_wait_warp(drain_bar, 0, kSitePvDone, &never);
   } else if (warp >= 4) {
     // ---------------------------- softmax, tile q -----------------------------
     if constexpr (NQ == 2) regs_inc<192>();
@@ -242,61 +250,53 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t o_tmem = tmem + q * C::QCOLS + C::SBUF * BN + lane_off;
+    const uint32_t s_tmem = tmem + q * C::QCOLS + C::TM_S + lane_off;
+    const uint32_t p_tmem = tmem + q * C::QCOLS + C::TM_P + lane_off;
+    const uint32_t o_tmem = tmem + q * C::QCOLS + C::TM_O + lane_off;
     const float c = p.c;
-    // V's padding column D is set to 1 in every tile, so column D of O
-    // accumulates the row sum of P in fp32 on the tensor core.
-    constexpr int TAIL = D - 64 * (C::DSLABS - 1);           // columns of V's last slab
-    const uint32_t one16 = BF16 ? 0x3F80u : 0x3C00u;
     uint32_t t = 0;        // tiles seen by this query-tile slot (all units)
-    uint32_t kvt = 0;      // key tiles seen (stage index)
     bool live = true;
     for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
       const int bh = u / p.tph, qg = u % p.tph;
       const int row = (qg * NQ + q) * 128 + r;
       float m_used = -INFINITY, rawmax = -INFINITY;
-      for (int j = 0; j < p.nkv; ++j, ++t, ++kvt) {
-        const uint32_t slot = t % C::SBUF, n = t / C::SBUF;
-        if (q == 0) {
-          // ones column of this tile's V rows (after the tile has landed)
-          const uint32_t st = kvt % C::STAGES, ns = kvt / C::STAGES;
-          live = __all_sync(0xffffffffu, mbar_wait(&v_full[st], ns & 1, kSiteVFull, abort_flag));
-          if (!live) break;
-          if (r < BN) {
-            uint8_t* vrow = sKV + st * C::STAGE + C::K_BYTES + (C::DSLABS - 1) * C::KV_SLAB + r * 128;
-            *reinterpret_cast<uint4*>(vrow + (((TAIL / 8) ^ (r & 7)) << 4)) = make_uint4(one16, 0u, 0u, 0u);
-            fence_proxy_async_smem();
-          }
-        }
-        live = __all_sync(0xffffffffu, mbar_wait(&s_full[q * C::SBUF + slot], n & 1, kSiteSFull, abort_flag));
+      for (int j = 0; j < p.nkv; ++j, ++t) {
+        live = __all_sync(0xffffffffu, mbar_wait(s_full, t & 1, kSiteSFull, abort_flag));
         if (!live) break;
         tc_fence_after();
-        const uint32_t s_tmem = tmem + q * C::QCOLS + slot * BN + lane_off;
         uint32_t v[BN];
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_x32(s_tmem + cc * 32, v + cc * 32);
         tmem_wait_ld();
         reg_fence<BN>(v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
         const int valid = p.M - j * BN;
         if (valid < BN) {
 #pragma unroll
           for (int k = 0; k < BN; ++k)
             if (k >= valid) v[k] = __float_as_uint(-INFINITY);
         }
-        // row max: eight independent three-input chains, then a small tree
-        float acc[8];
+        // row max: MAXCH independent three-input chains, then a small tree
+        constexpr int MAXCH = 16;
+        float acc[MAXCH];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(v[i]);
-        int k0 = 8;
+        for (int i = 0; i < MAXCH; ++i) acc[i] = __uint_as_float(v[i]);
+        int k0 = MAXCH;
 #pragma unroll
-        for (; k0 + 16 <= BN; k0 += 16)
+        for (; k0 + 2 * MAXCH <= BN; k0 += 2 * MAXCH)
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            acc[i] = fmax3(acc[i], __uint_as_float(v[k0 + i]), __uint_as_float(v[k0 + 8 + i]));
+          for (int i = 0; i < MAXCH; ++i)
+            acc[i] = fmax3(acc[i], __uint_as_float(v[k0 + i]), __uint_as_float(v[k0 + MAXCH + i]));
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < MAXCH; ++i)
           if (k0 + i < BN) acc[i] = fmaxf(acc[i], __uint_as_float(v[k0 + i]));
-        const float mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7])));
+#pragma unroll
+        for (int w = MAXCH; w > 1; w /= 2)
+#pragma unroll
+          for (int i = 0; i < w / 2; ++i) acc[i] = fmaxf(acc[i], acc[i + w / 2]);
+        const float mx = acc[0];
         rawmax = fmaxf(rawmax, mx);
         const float mt = mx * c;
         float alpha = 1.f;
@@ -323,11 +323,9 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           }
           pk[k] = pack2<BF16>(e0, e1);
         }
-#pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) tmem_st_x16(s_tmem + cc * 16, pk + cc * 16);
         if (j > 0) {
-          // P V of the previous tile must be done before O is touched
-          live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
+          // P V of the previous tile must be done: P is reused and O may be rescaled
+          live = __all_sync(0xffffffffu, mbar_wait(pv_done, (t - 1) & 1, kSitePvDone, abort_flag));
           if (!live) break;
           tc_fence_after();
           if (__any_sync(0xffffffffu, rescale)) {
@@ -344,14 +342,16 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
             }
           }
         }
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_st_x16(p_tmem + cc * 16, pk + cc * 16);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[q]);
+        if (lane == 0) mbar_arrive(p_full);
       }
       if (!live) break;
       // ---- epilogue: O / l, with l = column D of O ----
-      live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
+      live = __all_sync(0xffffffffu, mbar_wait(pv_done, (t - 1) & 1, kSitePvDone, abort_flag));
       if (!live) break;
       tc_fence_after();
       float l;

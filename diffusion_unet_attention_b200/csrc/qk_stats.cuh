@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
-    if (lane == 0) {
+    {   // the whole warp runs the loop; one elected lane issues
       constexpr uint32_t idesc = idesc_f16(128, 128, BF16, false, false);
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
       uint32_t kc = 0, ac = 0, ui = 0;
@@ -171,13 +171,13 @@ __global__ void __launch_bounds__(192, 1)
       for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
         int bh, rt, sp, cb0, cb1;
         qk_decode(p, u, bh, rt, sp, cb0, cb1);
-        if (!mbar_wait(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
+        if (!mbar_wait_warp(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
         tc_fence_after();
         for (int cb = cb0; cb < cb1; ++cb, ++kc, ++ac) {
           const uint32_t st = kc % C::KSTAGES, n = kc / C::KSTAGES;
           const uint32_t ab = ac & 1, na = ac >> 1;
-          if (!mbar_wait(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
-          if (!mbar_wait(&acc_empty[ab], (na & 1) ^ 1, kSiteAccEmpty, abort_flag)) { live = false; break; }
+          if (!mbar_wait_warp(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait_warp(&acc_empty[ab], (na & 1) ^ 1, kSiteAccEmpty, abort_flag)) { live = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem + ab * 128;
 #pragma unroll
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(192, 1)
       // Wait until every MMA this thread issued has finished.
       volatile uint32_t never = 0;
       mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kSiteAccFull, &never);
+      mbar_wait_warp(drain_bar, 0, kSiteAccFull, &never);
     }
   } else {
     // ------------------------------ epilogue ----------------------------------

@@ -240,10 +240,13 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   const int nsm = sm_count(dev);
   const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
   const uint64_t N = d->N, M = d->M;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mvt;
   if (!make_map_3d(&mq, Q, elem_type(d), D, N, bh, D * 2, N * D * 2, 64, 128)) return SDATTN_ERR_CUDA;
   if (!make_map_3d(&mk, K, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, BN)) return SDATTN_ERR_CUDA;
   if (!make_map_3d(&mv, V, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, BN)) return SDATTN_ERR_CUDA;
+  // V's last column slab is loaded only up to column D, keeping the padding
+  // (where the kernel keeps its ones column) untouched
+  if (!make_map_3d(&mvt, V, elem_type(d), D, M, bh, D * 2, M * D * 2, C::TAIL, BN)) return SDATTN_ERR_CUDA;
 
   FlashParams p;
   p.N = d->N;
@@ -257,7 +260,7 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   p.O = O;
   p.LS = LS;
   const int grid = p.units < nsm ? p.units : nsm;
-  kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+  kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, mv, mvt, p);
   return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
@@ -273,8 +276,7 @@ sdattn_status dispatch_flash(const sdattn_desc* d, const void* Q, const void* K,
       return two ? launch_flash<40, 2, 128, BF16>(d, Q, K, V, O, LS, s)
                  : launch_flash<40, 1, 128, BF16>(d, Q, K, V, O, LS, s);
     case 80:
-      return two ? launch_flash<80, 2, 128, BF16>(d, Q, K, V, O, LS, s)
-                 : launch_flash<80, 1, 128, BF16>(d, Q, K, V, O, LS, s);
+      return launch_flash<80, 1, 128, BF16>(d, Q, K, V, O, LS, s);
     case 160:
       return launch_flash<160, 1, 64, BF16>(d, Q, K, V, O, LS, s);
   }

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer --------------------------------
-    if (lane == 0) {
+    {   // the whole warp runs the loop; one elected lane issues
       constexpr uint32_t idesc = idesc_f16(128, C::PVN, BF16, false, true);
       const uint32_t v_base = smem_u32(sV);
       uint32_t c = 0, pc = 0;
@@ -143,8 +143,8 @@ __global__ void __launch_bounds__(192, 1)
         for (int kb = 0; kb < p.nkb; ++kb, ++c, ++pc) {
           const uint32_t st = c % C::STAGES, n = c / C::STAGES;
           const uint32_t pb = pc & 1, np = pc >> 1;
-          if (!mbar_wait(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
-          if (!mbar_wait(&p_full[pb], np & 1, kSitePFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait_warp(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait_warp(&p_full[pb], np & 1, kSitePFull, abort_flag)) { live = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       volatile uint32_t never = 0;
       mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kSiteOFull, &never);
+      mbar_wait_warp(drain_bar, 0, kSiteOFull, &never);
     }
   } else {
     // --------------------- softmax rows and epilogue --------------------------
