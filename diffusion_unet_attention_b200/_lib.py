@@ -27,7 +27,7 @@ STATUS = {
 
 # Every symbol include/sdattn.h declares.
 EXPORTS = ("sdattn_a_ld", "sdattn_workspace_bytes", "sdattn_qk_stats", "sdattn_softmax_av", "sdattn_flash",
-           "sdattn_device_error", "sdattn_status_string", "sdattn_version")
+           "sdattn_qk_stats_noalloc", "sdattn_device_error", "sdattn_status_string", "sdattn_version")
 
 
 class Desc(ctypes.Structure):
@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH):
     lib.sdattn_softmax_av.restype = ctypes.c_int
     lib.sdattn_flash.argtypes = [dp, vp, vp, vp, vp, vp, vp]
     lib.sdattn_flash.restype = ctypes.c_int
+    lib.sdattn_qk_stats_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
+    lib.sdattn_qk_stats_noalloc.restype = ctypes.c_int
     lib.sdattn_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sdattn_device_error.restype = ctypes.c_int
     lib.sdattn_status_string.argtypes = [ctypes.c_int]

@@ -286,6 +286,42 @@ sdattn_status dispatch_flash(const sdattn_desc* d, const void* Q, const void* K,
 }  // namespace
 
 // ============================================================================
+// Allocation-free variant of sdattn_qk_stats (no counterpart in the paper).
+//
+// Some callers cannot allocate device memory for a workspace: code that runs
+// inside a framework whose allocator it may not touch, plug-ins handed only
+// input and output buffers, or processes whose memory budget is fixed up front.
+// For them the split-reduction scratch of qk_stats lives in this file-scope
+// device array instead.  Every GPU that loads this library keeps the array
+// (kNoAllocScratchBytes) for the life of the process.
+// ============================================================================
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;   // 2 MiB
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// In host code `g_noalloc_scratch` only names the symbol; the device address
+// of the array is looked up once per device, with that device current.
+bool noalloc_scratch(int dev, void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return true;
+}
+
+}  // namespace
+
+// ============================================================================
 // C ABI
 // ============================================================================
 extern "C" {
@@ -358,6 +394,35 @@ sdattn_status sdattn_device_error(uint32_t* detail) {
   if (v != 0 && cudaMemcpyToSymbol(sdattn::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SDATTN_ERR_CUDA;
   if (detail) *detail = v;
   return v ? SDATTN_ERR_TIMEOUT : SDATTN_OK;
+}
+
+sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc* desc, const void* Q, const void* K, float* A, float* LS,
+                                      void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !A || !LS) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(A) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
+  // Same work split as sdattn_qk_stats; a single split uses no scratch at all.
+  const int dev = current_device();
+  const QKPlan pl = plan_qk(desc, sm_count(dev < 0 ? 0 : dev));
+  const int64_t tiles = static_cast<int64_t>(desc->B) * desc->H * pl.nrt;
+  const size_t need =
+      pl.nsplit > 1 ? ws_tickets_bytes(desc) + static_cast<size_t>(tiles) * 128 * pl.nsplit * sizeof(float2) : 0;
+  if (need > kNoAllocScratchBytes) return SDATTN_ERR_WORKSPACE;
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  void* ws = nullptr;
+  if (!noalloc_scratch(dev, &ws)) return SDATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The arrival counters must start at zero; the partials are overwritten.
+  if (pl.nsplit > 1 && cudaMemsetAsync(ws, 0, ws_tickets_bytes(desc), s) != cudaSuccess) return SDATTN_ERR_CUDA;
+  const bool bf = desc->dtype == SDATTN_BF16;
+  switch (desc->d) {
+    case 40: return bf ? launch_qk<40, true>(desc, Q, K, A, LS, ws, s) : launch_qk<40, false>(desc, Q, K, A, LS, ws, s);
+    case 80: return bf ? launch_qk<80, true>(desc, Q, K, A, LS, ws, s) : launch_qk<80, false>(desc, Q, K, A, LS, ws, s);
+    case 160:
+      return bf ? launch_qk<160, true>(desc, Q, K, A, LS, ws, s) : launch_qk<160, false>(desc, Q, K, A, LS, ws, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
 }
 
 const char* sdattn_status_string(sdattn_status status) {

@@ -125,6 +125,26 @@ sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const f
 sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K,
                            const void *V, void *O, float *LS_or_null, void *stream);
 
+/* Allocation-free variant of sdattn_qk_stats.  It has no counterpart in the
+ * paper; it exists for callers that cannot allocate device memory (for
+ * instance code running under a framework that owns the allocator, or a
+ * plug-in that is handed only its input and output buffers).
+ * Same inputs, outputs and results as sdattn_qk_stats, but the scratch of the
+ * split reduction is a 2 MiB array inside the library, present on every GPU
+ * that loads it until the process exits.  The call allocates nothing and
+ * calls no allocating routine.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture on the device.
+ *  - Each call clears the part of the array that must start at zero.  All
+ *    calls share the one array, which keeps the last call's contents, so calls
+ *    that may overlap on the GPU (different streams, different threads) race
+ *    and must not be issued; order them on one stream.
+ *  - Shapes whose split scratch would exceed 2 MiB return
+ *    SDATTN_ERR_WORKSPACE (use sdattn_qk_stats with a caller workspace). */
+sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc *desc, const void *Q, const void *K,
+                                      float *A, float *LS, void *stream);
+
 /* Reads and clears this device's error word (synchronises the device).
  * Returns SDATTN_OK, SDATTN_ERR_TIMEOUT, or SDATTN_ERR_CUDA if it cannot be
  * read.  If detail is not NULL it receives a code naming the wait that ran
