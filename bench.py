@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["sdattn", "reference"], default="sdattn")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-side", action="store_true",
+                    help="time the step set only (no per-form, per-kernel or end-to-end extras)")
     ap.add_argument("--case", default=None,
                     help="FORM:CONFIG, e.g. flash:2 -- run one form on one configuration (for profilers)")
     ap.add_argument("--reps", type=int, default=3)
@@ -301,7 +303,7 @@ def run_gpu(args, rank, world, local_rank):
 
     extra = {}
     e2e = None
-    if rank == 0:
+    if rank == 0 and not args.no_side:
         extra = side_measurements(torch, sd, stream, sets, scratch, issue, K=min(K, 50))
         e2e = end_to_end(torch, sd, stream, sets[0], scratch, steps=min(K, 10))
 
@@ -436,36 +438,52 @@ def end_to_end(torch, sd, stream, stepset, scratch, steps):
 # ----------------------------------------------------------------------------
 # CPU oracle (baseline leg and reference arm)
 # ----------------------------------------------------------------------------
-def oracle_sample(row_stride: int, seed_offset: int = 0):
-    """Runs the fp64 oracle on every `row_stride`-th query row of every call of
-    the step set; returns (algorithmic FLOPs done, seconds, threads)."""
-    import oracle
-    lib = oracle.load()
-    flops, secs = 0, 0.0
-    for ci, call in enumerate(CALLS):
-        q, k, v = synth.make_qkv(call, synth.STEP_SET_ID + seed_offset, call_id=ci)
-        qs = np.ascontiguousarray(q[:, :, ::row_stride])
+class OracleSample:
+    """The fp64 oracle on every `row_stride`-th query row of every call of the
+    step set.  Inputs are drawn and widened to fp64 once; `run()` times only
+    the oracle itself."""
+
+    _inputs = None
+
+    def __init__(self, row_stride: int):
+        import oracle
+        self.oracle = oracle
+        self.lib = oracle.load()
+        if OracleSample._inputs is None:
+            cache = []
+            for ci, call in enumerate(CALLS):
+                q, k, v = synth.make_qkv(call, synth.STEP_SET_ID, call_id=ci)
+                cache.append((call, q, np.ascontiguousarray(k, np.float64), np.ascontiguousarray(v, np.float64)))
+            OracleSample._inputs = cache
+        self.work = []
+        self.flops = 0
+        for call, q, k, v in OracleSample._inputs:
+            qs = np.ascontiguousarray(q[:, :, ::row_stride], np.float64)
+            self.work.append((qs, k, v, 1.0 / math.sqrt(call.d)))
+            self.flops += 4 * call.B * call.H * qs.shape[2] * call.M * call.d
+        self.stride = row_stride
+
+    def run(self) -> float:
         t = time.perf_counter()
-        oracle.attention(qs, k, v, 1.0 / math.sqrt(call.d), lib=lib)
-        secs += time.perf_counter() - t
-        flops += 4 * call.B * call.H * qs.shape[2] * call.M * call.d
-    return flops, secs, oracle.max_threads()
+        for qs, k, v, scale in self.work:
+            self.oracle.attention(qs, k, v, scale, lib=self.lib)
+        return time.perf_counter() - t
 
 
 def choose_stride(budget_s: float) -> int:
     """Row stride whose oracle sample takes about budget_s seconds."""
-    f, s, _ = oracle_sample(4096)
-    rate = f / max(s, 1e-6)
-    want = budget_s * rate
-    return max(1, int(STEP_FLOPS / max(want, 1.0)))
+    probe = OracleSample(256)
+    rate = probe.flops / max(probe.run(), 1e-6)
+    return max(1, int(round(STEP_FLOPS * 1.0 / max(budget_s * rate, 1.0))))
 
 
 def cpu_baseline(seconds: float):
-    stride = choose_stride(seconds)
-    f, s, thr = oracle_sample(stride)
-    return {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-            "sample": f"every {stride}-th query row of all 32 calls of the step set "
-                      f"({f / 1e9:.2f} GFLOP of the {STEP_FLOPS / 1e9:.1f} GFLOP step), fp64 C + OpenMP",
+    sample = OracleSample(choose_stride(seconds))
+    s = sample.run()
+    return {"value": round(sample.flops / s / 1e12, 6), "unit": "TFLOP/s", "cores": sample.oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"every {sample.stride}-th query row of all 32 calls of the step set "
+                      f"({sample.flops / 1e9:.2f} GFLOP of the {STEP_FLOPS / 1e9:.1f} GFLOP step), fp64 C + OpenMP",
             "seconds": round(s, 2)}
 
 
@@ -474,22 +492,22 @@ def run_reference(args, rank, world):
         return
     K, W = args.steps, args.warmup
     budget = 90.0 / max(K + W, 1)          # whole run about a minute and a half
-    stride = choose_stride(budget)
+    sample = OracleSample(choose_stride(budget))
     for _ in range(W):
-        oracle_sample(stride)
-    tot_f, tot_s, thr = 0, 0.0, 1
+        sample.run()
+    tot_s = 0.0
     for _ in range(K):
-        f, s, thr = oracle_sample(stride)
-        tot_f += f
-        tot_s += s
-    value = tot_f / tot_s / 1e12
+        tot_s += sample.run()
+    value = sample.flops * K / tot_s / 1e12
+    thr = sample.oracle.max_threads()
     line = {"metric": "attention us & TFLOP/s per UNet-step set (1xB200); % of tensor / HBM roofline",
             "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": round(STEP_FLOPS / (value * 1e12) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD}, "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                             "sample": f"every {stride}-th query row of all 32 calls per step"},
+                             "sample": f"every {sample.stride}-th query row of all 32 calls per step "
+                                       f"({sample.flops / 1e9:.3f} GFLOP per step)"},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

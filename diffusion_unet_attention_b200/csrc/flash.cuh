@@ -43,6 +43,7 @@ struct FlashParams {
   float scale;
   void* O;
   float* LS;   // optional
+  int inject_stall;   // test hook: the MMA warp first waits on a barrier nothing completes
 };
 
 template <int D, int NQ, int BN>
@@ -68,7 +69,7 @@ struct FlashCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = NQ * Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
-  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1;
+  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 2;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
   static_assert(STAGES >= 2, "key/value ring too shallow");
@@ -100,7 +101,8 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   uint64_t* p_full = s_free + 1;             // softmax -> MMA: P written (O rescaled)
   uint64_t* pv_done = p_full + 1;            // MMA -> softmax: P V done, P buffers free
   uint64_t* drain_bar = pv_done + 1;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* stall_bar = drain_bar + 1;       // never completed: target of the stall test hook
+  uint32_t* misc = reinterpret_cast<uint32_t*>(stall_bar + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -119,6 +121,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     mbar_init(p_full, 4 * NQ);
     mbar_init(pv_done, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(stall_bar, 1);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -200,6 +203,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV) + C::K_BYTES, C::KV_SLAB, 1024);
     uint32_t t_base = 0, kv_base = 0, ui = 0;
     bool live = true;
+    if (p.inject_stall) live = mbar_wait_warp(stall_bar, 0, kSiteInjected, abort_flag);   // runs out
     for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
       if (!mbar_wait_warp(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
       for (int j = 0; j <= p.nkv; ++j) {

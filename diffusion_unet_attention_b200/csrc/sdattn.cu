@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <mutex>
 
@@ -259,6 +260,11 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   p.c = d->scale * 1.4426950408889634f;
   p.O = O;
   p.LS = LS;
+  // Test hook for the bounded-wait path: with SDATTN_TEST_INJECT_STALL=1 in
+  // the environment, one wait in the kernel can never complete, runs out after
+  // about a second, and the call's results are left unwritten.
+  const char* stall = std::getenv("SDATTN_TEST_INJECT_STALL");
+  p.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
   const int grid = p.units < nsm ? p.units : nsm;
   kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, mv, mvt, p);
   return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;

@@ -21,7 +21,7 @@ __device__ uint32_t g_error_word = 0;
 enum WaitSite : uint32_t {
   kSiteQFull = 1, kSiteQEmpty, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty,
   kSiteAccFull, kSiteAccEmpty, kSiteSFull, kSitePFull, kSitePEmpty, kSitePvDone,
-  kSiteAFull, kSiteAEmpty, kSiteOFull, kSiteTicket
+  kSiteAFull, kSiteAEmpty, kSiteOFull, kSiteTicket, kSiteInjected
 };
 
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // one second
