@@ -45,13 +45,14 @@ struct QKCfg {
   static constexpr int KSTEPS = (D + 15) / 16;    // K=16 MMA steps (zero-padded past D)
   static constexpr int SLAB = 128 * 128;          // one slab of a 128-row tile, bytes
   static constexpr int KSTAGES = DSLABS == 1 ? 4 : (DSLABS == 2 ? 3 : 2);
-  static constexpr int NSTG = 4;                  // 4 KB staging buffers per epilogue warp
+  static constexpr int QBUF = 2;                  // Q double-buffered: the next unit's Q loads early
+  static constexpr int NSTG = DSLABS == 3 ? 2 : 4;   // 4 KB staging buffers per epilogue warp
   static constexpr int STG = 4096;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + DSLABS * SLAB;
+  static constexpr int OFF_K = OFF_Q + QBUF * DSLABS * SLAB;
   static constexpr int OFF_STG = OFF_K + KSTAGES * DSLABS * SLAB;
   static constexpr int OFF_BAR = OFF_STG + 4 * NSTG * STG;
-  static constexpr int NBAR = 2 + 2 * KSTAGES + 4 + 1;
+  static constexpr int NBAR = 2 * QBUF + 2 * KSTAGES + 4 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;   // + misc words + alignment slack
   static constexpr int NTHREADS = 192;
   static constexpr uint32_t TMEM_COLS = 256;
@@ -90,9 +91,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sStg = smem + C::OFF_STG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
+  uint64_t* q_full = bars;                // [QBUF]
+  uint64_t* q_empty = q_full + C::QBUF;   // [QBUF]
+  uint64_t* k_full = q_empty + C::QBUF;
   uint64_t* k_empty = k_full + C::KSTAGES;
   uint64_t* acc_full = k_empty + C::KSTAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -104,8 +105,10 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int i = 0; i < C::QBUF; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
     for (int i = 0; i < C::KSTAGES; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -132,6 +135,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  // Everything above touched only this CTA's own resources; global inputs and
+  // outputs are used only once the previous kernel of the stream is complete.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -141,10 +148,12 @@ __global__ void __launch_bounds__(192, 1)
       for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
         int bh, rt, sp, cb0, cb1;
         qk_decode(p, u, bh, rt, sp, cb0, cb1);
-        if (!mbar_wait(q_empty, (nq & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
+        const uint32_t qb = nq % C::QBUF, qn = nq / C::QBUF;
+        if (!mbar_wait(&q_empty[qb], (qn & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
         ++nq;
-        mbar_arrive_expect_tx(q_full, C::DSLABS * C::SLAB);
-        for (int s = 0; s < C::DSLABS; ++s) tma_load_3d(sQ + s * C::SLAB, &tmQ, 64 * s, rt * 128, bh, q_full);
+        mbar_arrive_expect_tx(&q_full[qb], C::DSLABS * C::SLAB);
+        for (int s = 0; s < C::DSLABS; ++s)
+          tma_load_3d(sQ + (qb * C::DSLABS + s) * C::SLAB, &tmQ, 64 * s, rt * 128, bh, &q_full[qb]);
         for (int cb = cb0; cb < cb1; ++cb, ++kc) {
           const uint32_t st = kc % C::KSTAGES, n = kc / C::KSTAGES;
           if (!mbar_wait(&k_empty[st], (n & 1) ^ 1, kSiteKEmpty, abort_flag)) { live = false; break; }
@@ -155,7 +164,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       // Let every load this thread issued land before the CTA can exit.
       volatile uint32_t never = 0;
-      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, kSiteQFull, &never);
+      for (uint32_t qb = 0; qb < C::QBUF && qb < nq; ++qb) {
+        const uint32_t uses = (nq - qb + C::QBUF - 1) / C::QBUF;
+        mbar_wait(&q_full[qb], (uses - 1) & 1, kSiteQFull, &never);
+      }
       for (uint32_t st = 0; st < C::KSTAGES && st < kc; ++st) {
         const uint32_t uses = (kc - st + C::KSTAGES - 1) / C::KSTAGES;
         mbar_wait(&k_full[st], (uses - 1) & 1, kSiteKFull, &never);
@@ -171,7 +183,8 @@ __global__ void __launch_bounds__(192, 1)
       for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
         int bh, rt, sp, cb0, cb1;
         qk_decode(p, u, bh, rt, sp, cb0, cb1);
-        if (!mbar_wait_warp(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
+        const uint32_t qb = ui % C::QBUF, qn = ui / C::QBUF;
+        if (!mbar_wait_warp(&q_full[qb], qn & 1, kSiteQFull, abort_flag)) { live = false; break; }
         tc_fence_after();
         for (int cb = cb0; cb < cb1; ++cb, ++kc, ++ac) {
           const uint32_t st = kc % C::KSTAGES, n = kc / C::KSTAGES;
@@ -183,14 +196,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < C::KSTEPS; ++kk) {
             const uint32_t off = (kk >> 2) * C::SLAB + (kk & 3) * 32;
-            const uint64_t ad = sdesc_sw128(q_base + off, 16, 1024);
+            const uint64_t ad = sdesc_sw128(q_base + qb * C::DSLABS * C::SLAB + off, 16, 1024);
             const uint64_t bd = sdesc_sw128(k_base + st * C::DSLABS * C::SLAB + off, 16, 1024);
             mma_ss(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
           mma_commit(&k_empty[st]);
           mma_commit(&acc_full[ab]);
         }
-        if (live) mma_commit(q_empty);
+        if (live) mma_commit(&q_empty[qb]);
       }
       // Wait until every MMA this thread issued has finished.
       volatile uint32_t never = 0;

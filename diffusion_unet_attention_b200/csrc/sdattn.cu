@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "sdattn.h"
 
@@ -91,6 +92,24 @@ bool ensure_smem(Kern kern, int bytes, std::atomic<uint64_t>& done, int dev) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
   done.fetch_or(bit, std::memory_order_acq_rel);
   return true;
+}
+
+// Launch with programmatic stream serialisation: the kernel may begin its
+// prologue while the previous kernel of the stream drains (the kernels wait
+// for it before touching global memory).
+template <typename... KArgs, typename... Args>
+bool launch(void (*kern)(KArgs...), int grid, int block, int smem, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess;
 }
 
 // --------------------------------------------------------------------------
@@ -192,8 +211,7 @@ sdattn_status launch_qk(const sdattn_desc* d, const void* Q, const void* K, floa
   p.tickets = static_cast<uint32_t*>(ws);
   p.part = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + ws_tickets_bytes(d));
   const int grid = pl.units < nsm ? pl.units : nsm;
-  kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, ma, p);
-  return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
+  return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, ma, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
 template <int D, bool BF16>
@@ -224,8 +242,7 @@ sdattn_status launch_av(const sdattn_desc* d, const float* A, const float* LS, c
   p.LS = LS;
   p.O = O;
   const int grid = p.units < nsm ? p.units : nsm;
-  kern<<<grid, 192, C::SMEM, stream>>>(ma, mv, p);
-  return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
+  return launch(kern, grid, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
 template <int D, int NQ, int BN, bool BF16, int NPOLY = 3>
@@ -266,8 +283,7 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   const char* stall = std::getenv("SDATTN_TEST_INJECT_STALL");
   p.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
   const int grid = p.units < nsm ? p.units : nsm;
-  kern<<<grid, C::NTHREADS, C::SMEM, stream>>>(mq, mk, mv, mvt, p);
-  return cudaGetLastError() == cudaSuccess ? SDATTN_OK : SDATTN_ERR_CUDA;
+  return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, mv, mvt, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
 template <bool BF16>

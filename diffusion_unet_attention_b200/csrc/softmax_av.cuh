@@ -105,6 +105,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  // Everything above touched only this CTA's own resources; global inputs and
+  // outputs are used only once the previous kernel of the stream is complete.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
