@@ -46,7 +46,7 @@ struct QKCfg {
   static constexpr int SLAB = 128 * 128;          // one slab of a 128-row tile, bytes
   static constexpr int KSTAGES = DSLABS == 1 ? 4 : (DSLABS == 2 ? 3 : 2);
   static constexpr int QBUF = 2;                  // Q double-buffered: the next unit's Q loads early
-  static constexpr int NSTG = DSLABS == 3 ? 2 : 4;   // 4 KB staging buffers per epilogue warp
+  static constexpr int NSTG = DSLABS == 1 ? 8 : (DSLABS == 2 ? 4 : 2);   // 4 KB staging buffers per epilogue warp
   static constexpr int STG = 4096;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBUF * DSLABS * SLAB;

@@ -28,6 +28,7 @@ using sdattn::QKParams;
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplit = 16;
+constexpr int kMinBlocksPerSplit = 4;
 
 // --------------------------------------------------------------------------
 // Driver entry point for tensor-map encoding (no link-time libcuda dependency)
@@ -136,7 +137,9 @@ CUtensorMapDataType elem_type(const sdattn_desc* d) {
 }
 
 // Column splits of the statistics reduction: the smallest power of two that
-// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit.
+// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit,
+// and never below kMinBlocksPerSplit column blocks per split (each split
+// pays a partial write and an arrival, which a one-block split cannot hide).
 struct QKPlan {
   int nrt, nb, nsplit, cbs, units;
 };
@@ -153,7 +156,7 @@ QKPlan plan_qk(const sdattn_desc* d, int nsm) {
   };
   int ns = 1;
   const int cap = pl.nb < kMaxSplit ? pl.nb : kMaxSplit;
-  while (ns * 2 <= cap && eff(base * ns) < 0.9) ns *= 2;
+  while (ns * 2 <= cap && pl.nb / (ns * 2) >= kMinBlocksPerSplit && eff(base * ns) < 0.9) ns *= 2;
   pl.cbs = (pl.nb + ns - 1) / ns;
   pl.nsplit = (pl.nb + pl.cbs - 1) / pl.cbs;
   pl.units = static_cast<int>(base * pl.nsplit);

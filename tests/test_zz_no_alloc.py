@@ -70,9 +70,9 @@ def test_matches_workspace_entry_point_twice(B, H, N, M, d):
 
 
 def test_rejects_shapes_beyond_its_scratch():
-    # 149 row tiles of a 2048-key row split 16 ways need about 2.4 MB of partials
+    # 149 row tiles of an 8192-key row split 16 ways need about 2.4 MB of partials
     lib = _lib.load()
-    desc = _lib.Desc(1, 149, 128, 2048, 40, _lib.SDATTN_F16, 0.15811388)
+    desc = _lib.Desc(1, 149, 128, 8192, 40, _lib.SDATTN_F16, 0.15811388)
     p = torch.empty(16, dtype=torch.float32, device=DEV)
     st = lib.sdattn_qk_stats_noalloc(ctypes.byref(desc), p.data_ptr(), p.data_ptr(), p.data_ptr(), p.data_ptr(),
                                      None)
