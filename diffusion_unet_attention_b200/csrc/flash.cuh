@@ -69,7 +69,7 @@ struct FlashCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = NQ * Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
-  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 2;
+  static constexpr int NBAR = 2 + 3 * STAGES + 5 * NQ + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
   static_assert(STAGES >= 2, "key/value ring too shallow");
@@ -95,13 +95,14 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   uint64_t* k_full = bars + 2;
   uint64_t* v_full = k_full + C::STAGES;
   uint64_t* kv_empty = v_full + C::STAGES;
-  // The NQ query tiles advance in lockstep, so each handshake has one barrier:
-  uint64_t* s_full = kv_empty + C::STAGES;   // MMA -> softmax: S of every query tile ready
-  uint64_t* s_free = s_full + 1;             // softmax -> MMA: S loaded, buffers free
-  uint64_t* p_full = s_free + 1;             // softmax -> MMA: P written (O rescaled)
-  uint64_t* pv_done = p_full + 1;            // MMA -> softmax: P V done, P buffers free
-  uint64_t* drain_bar = pv_done + 1;
-  uint64_t* stall_bar = drain_bar + 1;       // never completed: target of the stall test hook
+  // Each query tile has its own MMA-issuing warp and its own handshakes; the
+  // tiles share only the Q load and the key/value stages.
+  uint64_t* s_full = kv_empty + C::STAGES;   // [NQ] MMA -> softmax: S ready
+  uint64_t* s_free = s_full + NQ;            // [NQ] softmax -> MMA: S loaded, buffer free
+  uint64_t* p_full = s_free + NQ;            // [NQ] softmax -> MMA: P written (O rescaled)
+  uint64_t* pv_done = p_full + NQ;           // [NQ] MMA -> softmax: P V done, P free
+  uint64_t* drain_bar = pv_done + NQ;        // [NQ]
+  uint64_t* stall_bar = drain_bar + NQ;      // never completed: target of the stall test hook
   uint32_t* misc = reinterpret_cast<uint32_t*>(stall_bar + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
@@ -110,17 +111,19 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, NQ);
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], NQ);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4 * NQ);
-    mbar_init(p_full, 4 * NQ);
-    mbar_init(pv_done, 1);
-    mbar_init(drain_bar, 1);
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&drain_bar[i], 1);
+    }
     mbar_init(stall_bar, 1);
     misc[1] = 0;
     fence_mbar_init();
@@ -193,18 +196,22 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         mbar_wait(&v_full[st], (uses - 1) & 1, kSiteVFull, &never);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer --------------------------------
+  } else if (warp >= 1 && warp <= NQ) {
+    // --------------------------- MMA issuer, tile q ---------------------------
     // The whole warp runs the loop; one elected lane issues.  Per key tile j:
-    // S_j for every query tile (once the softmax has loaded S_{j-1}), then
-    // P V for tile j-1 (once P_{j-1} is written).
+    // S_j (once the softmax has loaded S_{j-1}), then P V for tile j-1 (once
+    // P_{j-1} is written).  Warp 1 + q serves query tile q only.
     if constexpr (NQ == 2) regs_dec<120>();
+    const int q = warp - 1;
     constexpr uint32_t idesc_s = idesc_f16(128, BN, BF16, false, false);
     constexpr uint32_t idesc_pv = idesc_f16(128, C::PVN, BF16, false, true);
-    // descriptors of the first Q slab and of stage 0's K and V; others by address offset
-    const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    // descriptors of this tile's first Q slab and of stage 0's K and V; others by address offset
+    const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ) + q * C::Q_TILE, 16, 1024);
     const uint64_t k_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);
     const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV) + C::K_BYTES, C::KV_SLAB, 1024);
+    const uint32_t s_tm = tmem + q * C::QCOLS + C::TM_S;
+    const uint32_t p_tm = tmem + q * C::QCOLS + C::TM_P;
+    const uint32_t o_tm = tmem + q * C::QCOLS + C::TM_O;
     uint32_t t_base = 0, kv_base = 0, ui = 0;
     bool live = true;
     if (p.inject_stall) live = mbar_wait_warp(stall_bar, 0, kSiteInjected, abort_flag);   // runs out
@@ -215,32 +222,26 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           const uint32_t kv = kv_base + j, t = t_base + j;
           const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
           if (!mbar_wait_warp(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
-          if (t >= 1 && !mbar_wait_warp(s_free, (t - 1) & 1, kSiteSFull, abort_flag)) { live = false; break; }
+          if (t >= 1 && !mbar_wait_warp(&s_free[q], (t - 1) & 1, kSiteSFull, abort_flag)) { live = false; break; }
           tc_fence_after();
           const uint64_t kd = k_desc0 + ((st * C::STAGE) >> 4);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q)
-#pragma unroll
-            for (int kk = 0; kk < C::KSTEPS; ++kk)
-              mma_ss(tmem + q * C::QCOLS + C::TM_S,
-                     q_desc0 + ((q * C::Q_TILE + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                     kd + (((kk >> 2) * C::KV_SLAB + (kk & 3) * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
-          mma_commit(s_full);
+          for (int kk = 0; kk < C::KSTEPS; ++kk)
+            mma_ss(s_tm, q_desc0 + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                   kd + (((kk >> 2) * C::KV_SLAB + (kk & 3) * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
+          mma_commit(&s_full[q]);
         }
         if (j >= 1) {
           const uint32_t kv = kv_base + j - 1, t = t_base + j - 1;
           const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
           if (!mbar_wait_warp(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
-          if (!mbar_wait_warp(p_full, t & 1, kSitePFull, abort_flag)) { live = false; break; }
+          if (!mbar_wait_warp(&p_full[q], t & 1, kSitePFull, abort_flag)) { live = false; break; }
           tc_fence_after();
           const uint64_t vd = v_desc0 + ((st * C::STAGE) >> 4);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q)
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ts(tmem + q * C::QCOLS + C::TM_O, tmem + q * C::QCOLS + C::TM_P + kk * 8,
-                     vd + ((kk * 2048) >> 4), idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
-          mma_commit(pv_done);
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+          mma_commit(&pv_done[q]);
           mma_commit(&kv_empty[st]);
         }
       }
@@ -249,8 +250,8 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       kv_base += p.nkv;
     }
     volatile uint32_t never = 0;
-    mma_commit(drain_bar);
-    mbar_wait_warp(drain_bar, 0, kSitePvDone, &never);
+    mma_commit(&drain_bar[q]);
+    mbar_wait_warp(&drain_bar[q], 0, kSitePvDone, &never);
   } else if (warp >= 4) {
     // ---------------------------- softmax, tile q -----------------------------
     if constexpr (NQ == 2) regs_inc<192>();
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       const int row = (qg * NQ + q) * 128 + r;
       float m_used = -INFINITY, rawmax = -INFINITY;
       for (int j = 0; j < p.nkv; ++j, ++t) {
-        live = __all_sync(0xffffffffu, mbar_wait(s_full, t & 1, kSiteSFull, abort_flag));
+        live = __all_sync(0xffffffffu, mbar_wait(&s_full[q], t & 1, kSiteSFull, abort_flag));
         if (!live) break;
         tc_fence_after();
         uint32_t v[BN];
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         reg_fence<BN>(v);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (lane == 0) mbar_arrive(&s_free[q]);
         const int valid = p.M - j * BN;
         if (valid < BN) {
 #pragma unroll
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         }
         if (j > 0) {
           // P V of the previous tile must be done: P is reused and O may be rescaled
-          live = __all_sync(0xffffffffu, mbar_wait(pv_done, (t - 1) & 1, kSitePvDone, abort_flag));
+          live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
           if (!live) break;
           tc_fence_after();
           if (__any_sync(0xffffffffu, rescale)) {
@@ -355,11 +356,11 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[q]);
       }
       if (!live) break;
       // ---- epilogue: O / l, with l = column D of O ----
-      live = __all_sync(0xffffffffu, mbar_wait(pv_done, (t - 1) & 1, kSitePvDone, abort_flag));
+      live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
       if (!live) break;
       tc_fence_after();
       float l;
