@@ -58,7 +58,9 @@ struct FlashCfg {
   static constexpr int V_BYTES = DSLABS * KV_SLAB;
   static constexpr int V_TX = (DSLABS - 1) * KV_SLAB + TAIL * 2 * BN;   // bytes the V loads deliver
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int STAGES_FIT = (226 * 1024 - NQ * Q_TILE) / STAGE;
+  static constexpr int QBUF = 2;                  // Q tiles double-buffered across work units
+  // 227 KB per CTA, less alignment slack, barriers and the tensor-memory word
+  static constexpr int STAGES_FIT = (232448 - 1024 - 16 - 8 * 32 - QBUF * NQ * Q_TILE) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   // tensor memory per query tile: S (BN fp32), P (BN/2 columns of 16-bit pairs), O (PVN fp32)
   static constexpr uint32_t TM_S = 0;
@@ -67,9 +69,9 @@ struct FlashCfg {
   static constexpr int QCOLS = BN + BN / 2 + PVN;
   static constexpr uint32_t TMEM_COLS = NQ * QCOLS <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = NQ * Q_TILE;
+  static constexpr int OFF_KV = QBUF * NQ * Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
-  static constexpr int NBAR = 2 + 3 * STAGES + 5 * NQ + 1;
+  static constexpr int NBAR = 2 * QBUF + 3 * STAGES + 5 * NQ + 2;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
   static_assert(STAGES >= 2, "key/value ring too shallow");
@@ -90,9 +92,9 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sKV = smem + C::OFF_KV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
+  uint64_t* q_full = bars;                  // [QBUF]
+  uint64_t* q_empty = q_full + C::QBUF;     // [QBUF] released by every query tile's MMA warp
+  uint64_t* k_full = q_empty + C::QBUF;
   uint64_t* v_full = k_full + C::STAGES;
   uint64_t* kv_empty = v_full + C::STAGES;
   // Each query tile has its own MMA-issuing warp and its own handshakes; the
@@ -103,6 +105,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   uint64_t* pv_done = p_full + NQ;           // [NQ] MMA -> softmax: P V done, P free
   uint64_t* drain_bar = pv_done + NQ;        // [NQ]
   uint64_t* stall_bar = drain_bar + NQ;      // never completed: target of the stall test hook
+  uint64_t* stagger = stall_bar + 1;         // query tile 0 -> 1, once: start half a tile apart
   uint32_t* misc = reinterpret_cast<uint32_t*>(stall_bar + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
@@ -110,8 +113,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, NQ);
+    for (int i = 0; i < C::QBUF; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], NQ);
+    }
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       mbar_init(&drain_bar[i], 1);
     }
     mbar_init(stall_bar, 1);
+    mbar_init(stagger, 4);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -169,12 +175,14 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       bool live = true;
       for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
         const int bh = u / p.tph, qg = u % p.tph;
-        if (!mbar_wait(q_empty, (nq & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
+        const uint32_t qb = nq % C::QBUF, qn = nq / C::QBUF;
+        if (!mbar_wait(&q_empty[qb], (qn & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
         ++nq;
-        mbar_arrive_expect_tx(q_full, NQ * C::Q_TILE);
+        mbar_arrive_expect_tx(&q_full[qb], NQ * C::Q_TILE);
         for (int q = 0; q < NQ; ++q)
           for (int s = 0; s < C::DSLABS; ++s)
-            tma_load_3d(sQ + q * C::Q_TILE + s * 16384, &tmQ, 64 * s, (qg * NQ + q) * 128, bh, q_full);
+            tma_load_3d(sQ + (qb * NQ + q) * C::Q_TILE + s * 16384, &tmQ, 64 * s, (qg * NQ + q) * 128, bh,
+                        &q_full[qb]);
         for (int j = 0; j < p.nkv; ++j, ++kvc) {
           const uint32_t st = kvc % C::STAGES, n = kvc / C::STAGES;
           if (!mbar_wait(&kv_empty[st], (n & 1) ^ 1, kSiteKEmpty, abort_flag)) { live = false; break; }
@@ -189,7 +197,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         }
       }
       volatile uint32_t never = 0;
-      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, kSiteQFull, &never);
+      for (uint32_t qb = 0; qb < C::QBUF && qb < nq; ++qb) {
+        const uint32_t uses = (nq - qb + C::QBUF - 1) / C::QBUF;
+        mbar_wait(&q_full[qb], (uses - 1) & 1, kSiteQFull, &never);
+      }
       for (uint32_t st = 0; st < C::STAGES && st < kvc; ++st) {
         const uint32_t uses = (kvc - st + C::STAGES - 1) / C::STAGES;
         mbar_wait(&k_full[st], (uses - 1) & 1, kSiteKFull, &never);
@@ -206,7 +217,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     constexpr uint32_t idesc_s = idesc_f16(128, BN, BF16, false, false);
     constexpr uint32_t idesc_pv = idesc_f16(128, C::PVN, BF16, false, true);
     // descriptors of this tile's first Q slab and of stage 0's K and V; others by address offset
-    const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ) + q * C::Q_TILE, 16, 1024);
+    const uint64_t q_desc00 = sdesc_sw128(smem_u32(sQ) + q * C::Q_TILE, 16, 1024);
     const uint64_t k_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);
     const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV) + C::K_BYTES, C::KV_SLAB, 1024);
     const uint32_t s_tm = tmem + q * C::QCOLS + C::TM_S;
@@ -216,7 +227,9 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     bool live = true;
     if (p.inject_stall) live = mbar_wait_warp(stall_bar, 0, kSiteInjected, abort_flag);   // runs out
     for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
-      if (!mbar_wait_warp(q_full, ui & 1, kSiteQFull, abort_flag)) { live = false; break; }
+      const uint32_t qb = ui % C::QBUF, qn = ui / C::QBUF;
+      if (!mbar_wait_warp(&q_full[qb], qn & 1, kSiteQFull, abort_flag)) { live = false; break; }
+      const uint64_t q_desc0 = q_desc00 + ((qb * NQ * C::Q_TILE) >> 4);
       for (int j = 0; j <= p.nkv; ++j) {
         if (j < p.nkv) {
           const uint32_t kv = kv_base + j, t = t_base + j;
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           mma_commit(&kv_empty[st]);
         }
       }
-      if (live) mma_commit(q_empty);
+      if (live) mma_commit(&q_empty[qb]);
       t_base += p.nkv;
       kv_base += p.nkv;
     }
@@ -265,6 +278,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     const float c = p.c;
     uint32_t t = 0;        // tiles seen by this query-tile slot (all units)
     bool live = true;
+    // The two query tiles run independently (own MMA warp, own handshakes,
+    // Q double-buffered); started half a tile apart, their softmax phases
+    // interleave on the SM instead of contending for the exponential unit.
+    if (NQ == 2 && q == 1) live = __all_sync(0xffffffffu, mbar_wait(stagger, 0, kSiteSFull, abort_flag));
     for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
       const int bh = u / p.tph, qg = u % p.tph;
       const int row = (qg * NQ + q) * 128 + r;
@@ -307,6 +324,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           for (int i = 0; i < w / 2; ++i) acc[i] = fmaxf(acc[i], acc[i + w / 2]);
         const float mx = acc[0];
         rawmax = fmaxf(rawmax, mx);
+        if (NQ == 2 && q == 0 && t == 0) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stagger);
+        }
         const float mt = mx * c;
         float alpha = 1.f;
         bool rescale = false;
