@@ -44,17 +44,19 @@ struct QKCfg {
   static constexpr int DSLABS = (D + 63) / 64;    // 64-element (128 B) column slabs of Q / K
   static constexpr int KSTEPS = (D + 15) / 16;    // K=16 MMA steps (zero-padded past D)
   static constexpr int SLAB = 128 * 128;          // one slab of a 128-row tile, bytes
-  static constexpr int KSTAGES = DSLABS == 1 ? 4 : (DSLABS == 2 ? 3 : 2);
+  static constexpr int KSTAGES = DSLABS == 1 ? 3 : 2;
   static constexpr int QBUF = 2;                  // Q double-buffered: the next unit's Q loads early
-  static constexpr int NSTG = DSLABS == 1 ? 8 : (DSLABS == 2 ? 4 : 2);   // 4 KB staging buffers per epilogue warp
+  static constexpr int EPI = DSLABS == 3 ? 1 : 2;   // epilogue warp groups (alternate 128-column blocks)
+  static constexpr int NSTG = DSLABS == 1 ? 4 : 2;   // 4 KB staging buffers per epilogue warp
   static constexpr int STG = 4096;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBUF * DSLABS * SLAB;
   static constexpr int OFF_STG = OFF_K + KSTAGES * DSLABS * SLAB;
-  static constexpr int OFF_BAR = OFF_STG + 4 * NSTG * STG;
+  static constexpr int OFF_MRG = OFF_STG + 4 * EPI * NSTG * STG;   // [2 slots][128 rows] float2
+  static constexpr int OFF_BAR = OFF_MRG + (EPI == 2 ? 2 * 128 * 8 : 0);
   static constexpr int NBAR = 2 * QBUF + 2 * KSTAGES + 4 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;   // + misc words + alignment slack
-  static constexpr int NTHREADS = 192;
+  static constexpr int NTHREADS = 64 + 128 * EPI;
   static constexpr uint32_t TMEM_COLS = 256;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -81,7 +83,7 @@ __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2)
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
     qk_stats_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const QKParams p) {
   using C = QKCfg<D>;
@@ -90,6 +92,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sStg = smem + C::OFF_STG;
+  float2* sMrg = reinterpret_cast<float2*>(smem + C::OFF_MRG);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;                // [QBUF]
   uint64_t* q_empty = q_full + C::QBUF;   // [QBUF]
@@ -215,16 +218,18 @@ __global__ void __launch_bounds__(192, 1)
     constexpr float L2E = 1.4426950408889634f;
     const int quarter = warp & 3;                 // TMEM lanes quarter*32 .. +31
     const int row_local = quarter * 32 + lane;    // row of the 128-row tile
+    const int e = (warp - 2) >> 2;                // epilogue group: with two, group e takes accumulator e
     uint8_t* stg = sStg + (warp - 2) * C::NSTG * C::STG;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    uint32_t ac = 0, sc = 0;
+    uint32_t ac = 0, sc = 0, ui = 0;
     bool live = true;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++ui) {
       int bh, rt, sp, cb0, cb1;
       qk_decode(p, u, bh, rt, sp, cb0, cb1);
       float m_run = -INFINITY, s_run = 0.f;
       for (int cb = cb0; cb < cb1 && live; ++cb, ++ac) {
         const uint32_t ab = ac & 1, na = ac >> 1;
+        if (C::EPI == 2 && static_cast<int>(ab) != e) continue;
         live = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], na & 1, kSiteAccFull, abort_flag));
         if (!live) break;
         tc_fence_after();
@@ -243,21 +248,33 @@ __global__ void __launch_bounds__(192, 1)
         const int col0 = cb * 128;
         const int valid = min(128, p.M - col0);
         // block partial (m_b, s_b) over the valid columns of this 128-column block
-        float mb = -INFINITY;
-        float sb = 0.f;
+        // eight independent chains for the max and for the sum, then a tree
+        float mx8[8], sm8[8];
         if (valid == 128) {
 #pragma unroll
-          for (int k = 0; k < 128; ++k) mb = fmaxf(mb, a[k]);
-          const float nmb = -mb * L2E;
+          for (int i = 0; i < 8; ++i) mx8[i] = fmax3(a[i], a[8 + i], a[16 + i]);
 #pragma unroll
-          for (int k = 0; k < 128; ++k) sb += ex2_approx(fmaf(a[k], L2E, nmb));
+          for (int k = 24; k < 128; k += 16)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], a[k + i], (k + 8 + i < 128) ? a[k + 8 + i] : a[k + i]);
         } else {
 #pragma unroll
-          for (int k = 0; k < 128; ++k) mb = (k < valid) ? fmaxf(mb, a[k]) : mb;
-          const float nmb = -mb * L2E;
+          for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < 128; ++k) sb += (k < valid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
+          for (int k = 0; k < 128; ++k) mx8[k & 7] = (k < valid) ? fmaxf(mx8[k & 7], a[k]) : mx8[k & 7];
         }
+        const float mb = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], fmax3(mx8[5], mx8[6], mx8[7])));
+        const float nmb = -mb * L2E;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
+        if (valid == 128) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) sm8[k & 7] += ex2_approx(fmaf(a[k], L2E, nmb));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) sm8[k & 7] += (k < valid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
+        }
+        const float sb = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
         ms_merge(m_run, s_run, mb, sb);
 
         // stream the block to A: 4 chunks of 32 columns x this warp's 32 rows
@@ -282,6 +299,15 @@ __global__ void __launch_bounds__(192, 1)
           ++sc;
         }
       }
+      // ---- the two groups' pairs merge; group 0 finishes the unit ----
+      if (C::EPI == 2) {
+        float2* slot = sMrg + (ui & 1) * 128;
+        if (e == 1) slot[row_local] = make_float2(m_run, s_run);
+        named_bar_sync(1, 256);
+        if (e == 1) continue;
+        const float2 o = slot[row_local];
+        ms_merge(m_run, s_run, o.x, o.y);
+      }
       // ---- unit result: the merged pair of this split ----
       const int row = rt * 128 + row_local;
       if (p.nsplit == 1) {
@@ -290,7 +316,7 @@ __global__ void __launch_bounds__(192, 1)
       } else {
         const int64_t tile = static_cast<int64_t>(bh) * p.nrt + rt;
         if (live) p.part[(tile * 128 + row_local) * p.nsplit + sp] = make_float2(m_run, s_run);
-        named_bar_sync(1, 128);
+        named_bar_sync(2, 128);
         if (threadIdx.x == 64) {
           uint32_t last = 0;
           if (live) {
@@ -299,7 +325,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           misc[2] = last;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(2, 128);
         if (misc[2]) {
           __threadfence();
           float m = -INFINITY, s = 0.f;
