@@ -109,6 +109,24 @@ def profiled_traffic():
 
 
 # ----------------------------------------------------------------------------
+# ranks: independent replicas; only the timing crosses processes
+# ----------------------------------------------------------------------------
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest `value` of all ranks (the job's time is its slowest rank's)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_step: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs the full step set (weak scaling)."""
+    return world * flops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
+# ----------------------------------------------------------------------------
 # clocks during the timed region
 # ----------------------------------------------------------------------------
 class ClockSampler:
@@ -294,12 +312,9 @@ def run_gpu(args, rank, world, local_rank):
     clk = clocks.stop()
     elapsed_ms = t0.elapsed_time(t1)
     dom_ms = sum(a.elapsed_time(b) for a, b in ev_dom) / (K * len(dom_calls))
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, device)
     ms_per_step = elapsed_ms / K
-    value = world * STEP_FLOPS * K / (elapsed_ms * 1e-3) / 1e12
+    value = job_throughput(world, STEP_FLOPS, K, elapsed_ms)
 
     extra = {}
     e2e = None
