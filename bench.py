@@ -208,7 +208,7 @@ class StepSet:
 
 
 class Scratch:
-    """A, LS and workspace shared by every partially fused call of a stream."""
+    """A, LS and workspace shared by every call of a stream."""
 
     def __init__(self, sd, torch, device, calls):
         self.sd, self.torch = sd, torch
@@ -223,7 +223,7 @@ class Scratch:
         sd = self.sd
         scale = 1.0 / math.sqrt(call.d)
         if form == "flash":
-            sd.flash(q, k, v, scale, out=o)
+            sd.flash(q, k, v, scale, out=o, ws=self.ws)
             return 1
         lda = (call.M + 3) // 4 * 4
         a = self.a[:call.B * call.H * call.N * lda].view(call.B, call.H, call.N, lda)
@@ -546,7 +546,7 @@ def run_case(args):
 
     def once():
         if form == "flash":
-            sd.flash(tq, tk, tv, scale, out=o)
+            sd.flash(tq, tk, tv, scale, out=o, ws=scratch.ws)
         elif form == "qk_stats":
             sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
         elif form == "softmax_av":

@@ -141,8 +141,13 @@ def softmax_av(a: torch.Tensor, ls: torch.Tensor, v: torch.Tensor, scale: float 
 
 
 def flash(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
-          out: torch.Tensor | None = None, return_ls: bool = False, out_ls: torch.Tensor | None = None):
-    """FlashAttention form.  Returns O [B,H,N,d] (and LS [B,H,N,2] if asked)."""
+          out: torch.Tensor | None = None, return_ls: bool = False, out_ls: torch.Tensor | None = None,
+          ws: torch.Tensor | None = None, use_workspace: bool = True):
+    """FlashAttention form.  Returns O [B,H,N,d] (and LS [B,H,N,2] if asked).
+
+    With a workspace (`ws`, else the cached one) the kernel may cut a block of
+    query rows' key range between two CTAs to even out its last wave;
+    `use_workspace=False` runs every block of rows whole."""
     B, H, N, M, d = _check_qk(q, k)
     if v.shape != k.shape or v.dtype != q.dtype or not v.is_cuda:
         raise ValueError("v must match k in shape and q in dtype")
@@ -154,8 +159,11 @@ def flash(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None
         LS = out_ls if out_ls is not None else torch.empty((B, H, N, 2), dtype=torch.float32, device=q.device)
         if LS.shape != (B, H, N, 2) or LS.dtype != torch.float32 or not LS.is_contiguous():
             raise ValueError("out_ls must be contiguous fp32 [B,H,N,2]")
+    w = (ws if ws is not None else workspace(desc, q.device)) if use_workspace else None
     st = _lib_handle().sdattn_flash(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), O.data_ptr(),
-                                    LS.data_ptr() if LS is not None else None, _stream(q.device))
+                                    LS.data_ptr() if LS is not None else None,
+                                    w.data_ptr() if w is not None else None, w.numel() if w is not None else 0,
+                                    _stream(q.device))
     _lib.check("sdattn_flash", st)
     return (O, LS) if (return_ls or out_ls is not None) else O
 
@@ -167,7 +175,13 @@ def partially_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: fl
 
 
 def device_error():
-    """(status name, detail code) of the device error word; reading clears it."""
+    """(status name, detail code) of the device error word; reading clears it.
+
+    After a timeout the cached workspaces are zero-filled anew, since the
+    abandoned calls may have left counters or partials in them."""
     detail = ctypes.c_uint32(0)
     st = _lib_handle().sdattn_device_error(ctypes.byref(detail))
+    if _lib.STATUS.get(st) == "SDATTN_ERR_TIMEOUT":
+        for ws in _workspaces.values():
+            ws.zero_()
     return _lib.STATUS.get(st, st), int(detail.value)

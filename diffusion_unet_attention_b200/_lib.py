@@ -64,7 +64,7 @@ def load(path: str = LIB_PATH):
     lib.sdattn_qk_stats.restype = ctypes.c_int
     lib.sdattn_softmax_av.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
     lib.sdattn_softmax_av.restype = ctypes.c_int
-    lib.sdattn_flash.argtypes = [dp, vp, vp, vp, vp, vp, vp]
+    lib.sdattn_flash.argtypes = [dp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.sdattn_flash.restype = ctypes.c_int
     lib.sdattn_qk_stats_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.sdattn_qk_stats_noalloc.restype = ctypes.c_int

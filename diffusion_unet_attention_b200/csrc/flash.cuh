@@ -8,7 +8,9 @@
 // register-intensive.
 //
 // B200 design.  One persistent CTA per SM walks (b*H + h, group of NQ
-// 128-row query tiles) units.  Roles:
+// 128-row query tiles) units, whole, or, when the units do not fill the last
+// wave, as equal shares of all (unit, key tile) pairs, a unit cut between two
+// CTAs being merged by the one that finishes second.  Roles:
 //   warp 0            TMA producer: the unit's NQ Q tiles, then a ring of
 //                     (K tile, V tile) stages, 128-byte swizzled, no multicast;
 //   warp 1            tcgen05 MMA issuer: S = Q K^T into tensor memory; once
@@ -44,6 +46,70 @@ struct FlashParams {
   void* O;
   float* LS;   // optional
   int inject_stall;   // test hook: the MMA warp first waits on a barrier nothing completes
+  // Split schedule (split != 0): CTA b of G = gridDim.x takes the contiguous
+  // range [b W / G, (b + 1) W / G) of the W = units * nkv (unit, key tile)
+  // pairs in unit-major order.  The host splits only when W / G >= nkv, so a
+  // unit is cut at most once, between two neighbouring CTAs: the head half
+  // (its first key tiles) ends CTA b's range, the tail half starts CTA b+1's.
+  // One of the two halves merges them, settled on a counter in `tickets`,
+  // from the other's partial rows in `part` (flash_cut_epilogue).  Without
+  // the split CTA b takes the whole units b, b + G, b + 2G, ...
+  int split;
+  uint32_t* tickets;   // [G * NQ], all zero on entry and on exit
+  float* part;         // [G * NQ][2][ROWF / 4][128 rows][4]: column quads, rows contiguous
+};
+
+// The work of one CTA as a list of segments: key tiles [j0, j1) of unit u.
+// Split schedule: a range [u_first:j_first, u_last:j_last) is walked as the
+// head half of unit u_last (its key tiles [0, j_last), when there is one)
+// first, then units u_first .. u_last - 1, the first from key tile j_first.
+// With the cut units first, both halves of a cut unit finish early in their
+// CTAs' runs and every CTA ends on a whole unit: the merge of two halves is
+// never the last thing a CTA does.
+struct FlashSegments {
+  int u, j0, j1;
+  int u_first, j_first, u_last;
+  __device__ __forceinline__ explicit FlashSegments(const FlashParams& p) {
+    if (p.split) {
+      const int64_t w = static_cast<int64_t>(p.units) * p.nkv;
+      const int64_t b = w * blockIdx.x / gridDim.x, e = w * (blockIdx.x + 1) / gridDim.x;
+      u_first = static_cast<int>(b / p.nkv);
+      j_first = static_cast<int>(b - static_cast<int64_t>(u_first) * p.nkv);
+      u_last = static_cast<int>(e / p.nkv);
+      const int j_last = static_cast<int>(e - static_cast<int64_t>(u_last) * p.nkv);
+      if (j_last > 0) {
+        u = u_last;
+        j0 = 0;
+        j1 = j_last;
+      } else {
+        first_whole(p);
+      }
+    } else {
+      u = blockIdx.x;
+      j0 = 0;
+      j1 = p.nkv;
+    }
+  }
+  __device__ __forceinline__ void first_whole(const FlashParams& p) {
+    u = u_first;
+    j0 = j_first;
+    j1 = u_first < u_last ? p.nkv : j0;
+  }
+  __device__ __forceinline__ bool valid(const FlashParams& p) const { return j0 < j1 && u < p.units; }
+  __device__ __forceinline__ void next(const FlashParams& p) {
+    if (p.split) {
+      if (u == u_last) {
+        first_whole(p);
+      } else {
+        ++u;
+        j0 = 0;
+        j1 = u < u_last ? p.nkv : 0;
+      }
+    } else {
+      u += gridDim.x;
+    }
+  }
+  __device__ __forceinline__ bool cut(const FlashParams& p) const { return j0 > 0 || j1 < p.nkv; }
 };
 
 template <int D, int NQ, int BN>
@@ -72,14 +138,149 @@ struct FlashCfg {
   static constexpr int OFF_KV = QBUF * NQ * Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
   static constexpr int NBAR = 2 * QBUF + 3 * STAGES + 5 * NQ + 2;
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static constexpr int MISC = 4 + 4 * NQ;   // words after the barriers
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + MISC * 4 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
+  // a partial row of a cut unit: D unnormalised O columns, then (m, l, raw max), padded to 16 bytes
+  static constexpr int ROWF = (D + 3 + 3) / 4 * 4;
   static_assert(STAGES >= 2, "key/value ring too shallow");
   static_assert(NQ * QCOLS <= 512, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
   static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
 };
+
+// A unit whose key range is cut between two CTAs (split schedule) is
+// finished by whichever half can see the other's results: each half has its
+// unnormalised rows O, running max m (base 2, scaled), row sum l and raw
+// score max, and the merge always combines head (h) then tail (t):
+//   m = max(m_h, m_t),  O = (O_h 2^(m_h-m) + O_t 2^(m_t-m)) / (l_h 2^(m_h-m) + l_t 2^(m_t-m)).
+// A half that cannot merge leaves its rows in the workspace, stored as quads
+// of columns with the 128 rows of a quad contiguous (32 consecutive rows
+// read or write 512 contiguous bytes):
+//   part[slot][half][ROWF / 4][128][4],  quad D / 4 = (m, l, raw max, 0).
+// Who merges is settled on one counter per (cut, query tile), by atomic adds
+// with acquire-release semantics:
+//   head: writes its rows, then adds 1;
+//   tail: adds 2 first; if the head's 1 is there it merges at once, without
+//         writing its rows; otherwise it writes them and adds 4;
+// the add that completes {1, 4} merges (the head, seeing 4; or the tail's
+// second add, seeing 1).  Exactly one side merges, from the other's rows in
+// the workspace and its own in tensor memory.  With each CTA's head half
+// scheduled first, the tail normally finds the head done.
+template <int ROWF>
+__device__ __forceinline__ float4* partial_rows(float* part, int64_t slot, int half) {
+  return reinterpret_cast<float4*>(part) + (slot * 2 + half) * (ROWF / 4) * 128;
+}
+
+// named barrier of query tile q's four softmax warps (ids fixed at compile time)
+__device__ __forceinline__ void softmax_bar_sync(int q) {
+  if (q == 0)
+    named_bar_sync(1, 128);
+  else
+    named_bar_sync(2, 128);
+}
+
+// One counter update for the tile: thread r == 0 adds v (acquire-release),
+// the old value reaches every thread of the tile through `flag`.
+__device__ __forceinline__ uint32_t tile_count(uint32_t* ticket, uint32_t v, int q, int r, volatile uint32_t* flag) {
+  if (r == 0) *flag = atomic_add_acq_rel_gpu(ticket, v);
+  softmax_bar_sync(q);
+  return *flag;
+}
+
+// Epilogue of a cut unit for the tile's 128 softmax threads (one row each).
+// flags: two words, used once each.  Out of line: it runs at most twice per
+// CTA, and inlined it would weigh on the register allocation of the softmax
+// loop (the softmax warps hold more registers than any callee may use).
+template <int D, bool BF16, int ROWF>
+__device__ __noinline__ void flash_cut_epilogue(float* part, uint32_t* tickets, float* LS, int N, float scale,
+                                                float c, uint32_t o_tmem, int side, int64_t slot, int q, int r,
+                                                int bh, int row, float m_used, float l, float rawmax,
+                                                volatile uint32_t* flags, uint8_t* orow) {
+  float4* mine = partial_rows<ROWF>(part, slot, side) + r;
+  const float4* theirs = partial_rows<ROWF>(part, slot, side ^ 1) + r;
+  constexpr int G = D / 8 < 5 ? D / 8 : 5;   // chunks of 8 columns per tensor-memory wait
+  static_assert((D / 8) % G == 0, "column groups");
+  auto write_mine = [&]() {
+#pragma unroll
+    for (int g0 = 0; g0 < D / 8; g0 += G) {
+      uint32_t o[8 * G];
+#pragma unroll
+      for (int i = 0; i < G; ++i) tmem_ld_x8(o_tmem + (g0 + i) * 8, o + 8 * i);
+      tmem_wait_ld();
+      reg_fence<8 * G>(o);
+#pragma unroll
+      for (int i = 0; i < 2 * G; ++i)
+        __stcg(mine + (g0 * 2 + i) * 128, make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                                     __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3])));
+    }
+    __stcg(mine + (D / 4) * 128, make_float4(m_used, l, rawmax, 0.f));
+    softmax_bar_sync(q);   // the tile's rows before the count that publishes them
+  };
+  bool merge, wrote = true;
+  if (side == 0) {
+    write_mine();
+    merge = (tile_count(&tickets[slot], 1u, q, r, &flags[0]) & 4u) != 0u;
+  } else {
+    merge = (tile_count(&tickets[slot], 2u, q, r, &flags[0]) & 1u) != 0u;
+    wrote = !merge;
+    if (!merge) {
+      write_mine();
+      merge = (tile_count(&tickets[slot], 4u, q, r, &flags[1]) & 1u) != 0u;
+    }
+  }
+  if (!merge) return;
+  const float4 t2 = __ldcg(theirs + (D / 4) * 128);
+  const float m_h = side ? t2.x : m_used, m_t = side ? m_used : t2.x;
+  const float l_h = side ? t2.y : l, l_t = side ? l : t2.y;
+  const float m = fmaxf(m_h, m_t);
+  const float a_h = ex2_approx(m_h - m), a_t = ex2_approx(m_t - m);
+  const float a_mine = side ? a_t : a_h, a_theirs = side ? a_h : a_t;
+  const float lsum = fmaf(l_h, a_h, l_t * a_t);
+  const float inv = 1.f / lsum;
+#pragma unroll
+  for (int g0 = 0; g0 < D / 8; g0 += G) {
+    uint32_t o[8 * G];
+    float4 u[2 * G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) tmem_ld_x8(o_tmem + (g0 + i) * 8, o + 8 * i);
+#pragma unroll
+    for (int i = 0; i < 2 * G; ++i) u[i] = __ldcg(theirs + (g0 * 2 + i) * 128);
+    tmem_wait_ld();
+    reg_fence<8 * G>(o);
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      const float g[8] = {u[2 * i].x, u[2 * i].y, u[2 * i].z, u[2 * i].w,
+                          u[2 * i + 1].x, u[2 * i + 1].y, u[2 * i + 1].z, u[2 * i + 1].w};
+      float f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float ov = __uint_as_float(o[8 * i + k]);
+        f[k] = (side ? fmaf(g[k], a_h, ov * a_mine) : fmaf(ov, a_h, g[k] * a_theirs)) * inv;
+      }
+      uint4 w;
+      w.x = pack2<BF16>(f[0], f[1]);
+      w.y = pack2<BF16>(f[2], f[3]);
+      w.z = pack2<BF16>(f[4], f[5]);
+      w.w = pack2<BF16>(f[6], f[7]);
+      if (row < N) *reinterpret_cast<uint4*>(orow + (g0 + i) * 16) = w;
+    }
+  }
+  if (LS != nullptr && row < N) {
+    const float raw = fmaxf(rawmax, t2.z);
+    *reinterpret_cast<float2*>(LS + 2 * (static_cast<int64_t>(bh) * N + row)) =
+        make_float2(raw * scale, lsum * ex2_approx(m - raw * c));
+  }
+  // leave the workspace all zero for the next call
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < ROWF / 4; ++k) {
+    if (wrote) __stcg(mine + k * 128, z);
+    __stcg(const_cast<float4*>(theirs) + k * 128, z);
+  }
+  if (r == 0) tickets[slot] = 0u;
+}
 
 template <int D, int NQ, int BN, bool BF16, int NPOLY>
 __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
@@ -106,7 +307,8 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
   uint64_t* drain_bar = pv_done + NQ;        // [NQ]
   uint64_t* stall_bar = drain_bar + NQ;      // never completed: target of the stall test hook
   uint64_t* stagger = stall_bar + 1;         // query tile 0 -> 1, once: start half a tile apart
-  uint32_t* misc = reinterpret_cast<uint32_t*>(stall_bar + 1);
+  // [0] tensor memory, [1] abort, [4 + 4q + 2k ..]: tile q's two count words for its k-th cut unit
+  uint32_t* misc = reinterpret_cast<uint32_t*>(stagger + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -173,8 +375,8 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     if (lane == 0) {
       uint32_t kvc = 0, nq = 0;
       bool live = true;
-      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
-        const int bh = u / p.tph, qg = u % p.tph;
+      for (FlashSegments sg(p); sg.valid(p) && live; sg.next(p)) {
+        const int bh = sg.u / p.tph, qg = sg.u % p.tph;
         const uint32_t qb = nq % C::QBUF, qn = nq / C::QBUF;
         if (!mbar_wait(&q_empty[qb], (qn & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
         ++nq;
@@ -183,7 +385,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           for (int s = 0; s < C::DSLABS; ++s)
             tma_load_3d(sQ + (qb * NQ + q) * C::Q_TILE + s * 16384, &tmQ, 64 * s, (qg * NQ + q) * 128, bh,
                         &q_full[qb]);
-        for (int j = 0; j < p.nkv; ++j, ++kvc) {
+        for (int j = sg.j0; j < sg.j1; ++j, ++kvc) {
           const uint32_t st = kvc % C::STAGES, n = kvc / C::STAGES;
           if (!mbar_wait(&kv_empty[st], (n & 1) ^ 1, kSiteKEmpty, abort_flag)) { live = false; break; }
           uint8_t* sK = sKV + st * C::STAGE;
@@ -226,12 +428,13 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     uint32_t t_base = 0, kv_base = 0, ui = 0;
     bool live = true;
     if (p.inject_stall) live = mbar_wait_warp(stall_bar, 0, kSiteInjected, abort_flag);   // runs out
-    for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
+    for (FlashSegments sg(p); sg.valid(p) && live; sg.next(p), ++ui) {
       const uint32_t qb = ui % C::QBUF, qn = ui / C::QBUF;
       if (!mbar_wait_warp(&q_full[qb], qn & 1, kSiteQFull, abort_flag)) { live = false; break; }
       const uint64_t q_desc0 = q_desc00 + ((qb * NQ * C::Q_TILE) >> 4);
-      for (int j = 0; j <= p.nkv; ++j) {
-        if (j < p.nkv) {
+      const int len = sg.j1 - sg.j0;
+      for (int j = 0; j <= len; ++j) {
+        if (j < len) {
           const uint32_t kv = kv_base + j, t = t_base + j;
           const uint32_t st = kv % C::STAGES, n = kv / C::STAGES;
           if (!mbar_wait_warp(&k_full[st], n & 1, kSiteKFull, abort_flag)) { live = false; break; }
@@ -259,8 +462,8 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         }
       }
       if (live) mma_commit(&q_empty[qb]);
-      t_base += p.nkv;
-      kv_base += p.nkv;
+      t_base += len;
+      kv_base += len;
     }
     volatile uint32_t never = 0;
     mma_commit(&drain_bar[q]);
@@ -282,11 +485,12 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     // Q double-buffered); started half a tile apart, their softmax phases
     // interleave on the SM instead of contending for the exponential unit.
     if (NQ == 2 && q == 1) live = __all_sync(0xffffffffu, mbar_wait(stagger, 0, kSiteSFull, abort_flag));
-    for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
-      const int bh = u / p.tph, qg = u % p.tph;
+    int kcut = 0;          // cut units seen (at most two)
+    for (FlashSegments sg(p); sg.valid(p) && live; sg.next(p)) {
+      const int bh = sg.u / p.tph, qg = sg.u % p.tph;
       const int row = (qg * NQ + q) * 128 + r;
       float m_used = -INFINITY, rawmax = -INFINITY;
-      for (int j = 0; j < p.nkv; ++j, ++t) {
+      for (int j = sg.j0; j < sg.j1; ++j, ++t) {
         live = __all_sync(0xffffffffu, mbar_wait(&s_full[q], t & 1, kSiteSFull, abort_flag));
         if (!live) break;
         tc_fence_after();
@@ -334,7 +538,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         if (mt > m_used + 8.f) {
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
-          rescale = (j > 0);
+          rescale = (j > sg.j0);
         }
         // p = 2^(s*c - m): NPOLY of every 8 pairs on the FMA pipe, the rest on MUFU
         const uint64_t c2 = f2_pack(c, c);
@@ -353,7 +557,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           }
           pk[k] = pack2<BF16>(e0, e1);
         }
-        if (j > 0) {
+        if (j > sg.j0) {
           // P V of the previous tile must be done: P is reused and O may be rescaled
           live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
           if (!live) break;
@@ -392,25 +596,33 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         reg_fence<8>(o);
         l = __uint_as_float(o[0]);
       }
-      const float inv = 1.f / l;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row) * D * 2;
+      if (!(p.split && sg.cut(p))) {
+        const float inv = 1.f / l;
 #pragma unroll
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        uint32_t o[8];
-        tmem_ld_x8(o_tmem + c8 * 8, o);
-        tmem_wait_ld();
-        reg_fence<8>(o);
-        uint4 w;
-        w.x = pack2<BF16>(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
-        w.y = pack2<BF16>(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
-        w.z = pack2<BF16>(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
-        w.w = pack2<BF16>(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
-        if (row < p.N) *reinterpret_cast<uint4*>(orow + c8 * 16) = w;
-      }
-      if (p.LS != nullptr && row < p.N) {
-        const float L = rawmax * p.scale;
-        const float S = l * ex2_approx(m_used - rawmax * c);
-        *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(L, S);
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          uint32_t o[8];
+          tmem_ld_x8(o_tmem + c8 * 8, o);
+          tmem_wait_ld();
+          reg_fence<8>(o);
+          uint4 w;
+          w.x = pack2<BF16>(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+          w.y = pack2<BF16>(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+          w.z = pack2<BF16>(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+          w.w = pack2<BF16>(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+          if (row < p.N) *reinterpret_cast<uint4*>(orow + c8 * 16) = w;
+        }
+        if (p.LS != nullptr && row < p.N) {
+          const float L = rawmax * p.scale;
+          const float S = l * ex2_approx(m_used - rawmax * c);
+          *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(L, S);
+        }
+      } else if (kcut < 2) {
+        const int side = sg.j0 > 0 ? 1 : 0;   // 0: head half, 1: tail half
+        flash_cut_epilogue<D, BF16, C::ROWF>(p.part, p.tickets, p.LS, p.N, p.scale, c, o_tmem, side,
+                                            static_cast<int64_t>(blockIdx.x - side) * NQ + q, q, r, bh, row, m_used,
+                                            l, rawmax, misc + 4 + 4 * q + 2 * kcut, orow);
+        ++kcut;
       }
       tc_fence_before();
     }

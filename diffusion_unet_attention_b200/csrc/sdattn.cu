@@ -170,11 +170,34 @@ size_t ws_tickets_bytes(const sdattn_desc* d) {
   return static_cast<size_t>((tiles * 4 + 255) / 256 * 256);
 }
 
-size_t ws_bytes(const sdattn_desc* d) {
+size_t qk_ws_bytes(const sdattn_desc* d) {
   const int64_t tiles = static_cast<int64_t>(d->B) * d->H * ((d->N + 127) / 128);
   const int nb = (d->M + 127) / 128;
   const int smax = nb < kMaxSplit ? nb : kMaxSplit;
   return ws_tickets_bytes(d) + static_cast<size_t>(tiles) * 128 * smax * sizeof(float2);
+}
+
+// Flash workspace, used when a unit's key range is cut between two CTAs:
+//   [tickets: one uint32 per (CTA, query tile), padded to 256 B]
+//   [partials: per (CTA, query tile, half, row) one row of ROWF floats]
+// sized for a grid of one CTA per SM and the most query tiles a CTA runs at d.
+int flash_nq_max(int d) { return d == 40 ? 2 : 1; }
+
+size_t flash_ws_tickets_bytes(const sdattn_desc* d, int nsm) {
+  return static_cast<size_t>((static_cast<int64_t>(nsm) * flash_nq_max(d->d) * 4 + 255) / 256 * 256);
+}
+
+size_t flash_ws_bytes(const sdattn_desc* d, int nsm) {
+  const int rowf = (d->d + 3 + 3) / 4 * 4;
+  return flash_ws_tickets_bytes(d, nsm) +
+         static_cast<size_t>(nsm) * flash_nq_max(d->d) * 2 * 128 * rowf * sizeof(float);
+}
+
+size_t ws_bytes(const sdattn_desc* d) {
+  const int dev = current_device();
+  const size_t qk = qk_ws_bytes(d);
+  const size_t fl = flash_ws_bytes(d, sm_count(dev < 0 ? 0 : dev));
+  return qk > fl ? qk : fl;
 }
 
 // --------------------------------------------------------------------------
@@ -250,7 +273,7 @@ sdattn_status launch_av(const sdattn_desc* d, const float* A, const float* LS, c
 
 template <int D, int NQ, int BN, bool BF16, int NPOLY = 3>
 sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
-                           cudaStream_t stream) {
+                           void* ws, cudaStream_t stream) {
   using C = FlashCfg<D, NQ, BN>;
   const int dev = current_device();
   if (dev < 0) return SDATTN_ERR_CUDA;
@@ -285,25 +308,34 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   // about a second, and the call's results are left unwritten.
   const char* stall = std::getenv("SDATTN_TEST_INJECT_STALL");
   p.inject_stall = (stall != nullptr && stall[0] == '1') ? 1 : 0;
+  // Whole units leave the last wave of CTAs part-empty when units is just
+  // above a multiple of the SM count; then (given a workspace) every CTA
+  // takes an equal share of the (unit, key tile) pairs instead, cutting at
+  // most one unit at each end of its range.
+  const int64_t waves = (p.units + nsm - 1) / nsm;
+  const double eff = static_cast<double>(p.units) / static_cast<double>(waves * nsm);
+  p.split = (ws != nullptr && p.units > nsm && p.nkv >= 2 && eff < 0.9) ? 1 : 0;
+  p.tickets = static_cast<uint32_t*>(ws);
+  p.part = ws ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flash_ws_tickets_bytes(d, nsm)) : nullptr;
   const int grid = p.units < nsm ? p.units : nsm;
   return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, mv, mvt, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
 template <bool BF16>
 sdattn_status dispatch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
-                             cudaStream_t s) {
+                             void* ws, cudaStream_t s) {
   const int dev = current_device();
   const int nsm = sm_count(dev < 0 ? 0 : dev);
   const int64_t pairs = static_cast<int64_t>(d->B) * d->H * ((d->N + 255) / 256);
   const bool two = pairs >= nsm;   // enough work for two query tiles per CTA
   switch (d->d) {
     case 40:
-      return two ? launch_flash<40, 2, 128, BF16>(d, Q, K, V, O, LS, s)
-                 : launch_flash<40, 1, 128, BF16>(d, Q, K, V, O, LS, s);
+      return two ? launch_flash<40, 2, 128, BF16>(d, Q, K, V, O, LS, ws, s)
+                 : launch_flash<40, 1, 128, BF16>(d, Q, K, V, O, LS, ws, s);
     case 80:
-      return launch_flash<80, 1, 128, BF16>(d, Q, K, V, O, LS, s);
+      return launch_flash<80, 1, 128, BF16>(d, Q, K, V, O, LS, ws, s);
     case 160:
-      return launch_flash<160, 1, 64, BF16>(d, Q, K, V, O, LS, s);
+      return launch_flash<160, 1, 64, BF16>(d, Q, K, V, O, LS, ws, s);
   }
   return SDATTN_ERR_UNSUPPORTED;
 }
@@ -367,7 +399,7 @@ sdattn_status sdattn_qk_stats(const sdattn_desc* desc, const void* Q, const void
   if (st != SDATTN_OK) return st;
   if (!Q || !K || !A || !LS) return SDATTN_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(A) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
-  if (!ws || ws_size < ws_bytes(desc)) return SDATTN_ERR_WORKSPACE;
+  if (!ws || ws_size < qk_ws_bytes(desc)) return SDATTN_ERR_WORKSPACE;
   if (!aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf = desc->dtype == SDATTN_BF16;
@@ -399,15 +431,21 @@ sdattn_status sdattn_softmax_av(const sdattn_desc* desc, const float* A, const f
 }
 
 sdattn_status sdattn_flash(const sdattn_desc* desc, const void* Q, const void* K, const void* V, void* O,
-                           float* LS_or_null, void* stream) {
+                           float* LS_or_null, void* ws, size_t ws_size, void* stream) {
   const sdattn_status st = check_desc(desc);
   if (st != SDATTN_OK) return st;
   if (!Q || !K || !V || !O) return SDATTN_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
   if (LS_or_null && !aligned16(LS_or_null)) return SDATTN_ERR_ALIGNMENT;
+  if (ws && !aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
+  if (!ws && ws_size != 0) return SDATTN_ERR_WORKSPACE;
+  if (ws) {
+    const int dev = current_device();
+    if (ws_size < flash_ws_bytes(desc, sm_count(dev < 0 ? 0 : dev))) return SDATTN_ERR_WORKSPACE;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return desc->dtype == SDATTN_BF16 ? dispatch_flash<true>(desc, Q, K, V, O, LS_or_null, s)
-                                    : dispatch_flash<false>(desc, Q, K, V, O, LS_or_null, s);
+  return desc->dtype == SDATTN_BF16 ? dispatch_flash<true>(desc, Q, K, V, O, LS_or_null, ws, s)
+                                    : dispatch_flash<false>(desc, Q, K, V, O, LS_or_null, ws, s);
 }
 
 sdattn_status sdattn_device_error(uint32_t* detail) {

@@ -248,7 +248,7 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 #define SD_R8(r, o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), \
                     "=r"(r[o + 4]), "=r"(r[o + 5]), "=r"(r[o + 6]), "=r"(r[o + 7])
 
-__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
+__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t* r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : SD_R8(r, 0)
                : "r"(taddr));
@@ -266,6 +266,17 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t* r) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Adds to a global counter with acquire-release semantics at GPU scope and
+// returns the old value.  The release makes the writes that happen before it
+// (this CTA's, when a barrier precedes it) visible to whoever later observes
+// the count; the acquire makes the writes released by earlier adders visible
+// to this thread (and, after a following barrier, to the CTA).
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
 
 // Ties registers written by an asynchronous tcgen05.ld to a point after
 // tcgen05.wait::ld, so the compiler cannot hoist their uses above the wait.

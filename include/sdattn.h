@@ -87,11 +87,12 @@ typedef enum {
  * Returns -1 for an invalid descriptor. */
 int64_t sdattn_a_ld(const sdattn_desc *desc);
 
-/* Bytes of workspace that sdattn_qk_stats and sdattn_softmax_av need for this
- * shape on the current device (split-reduction partials plus arrival
- * counters).  The same workspace serves both calls and any shape.  It must be
- * zero-filled once before its first use; every completed call leaves all of
- * it zero again.  After SDATTN_ERR_TIMEOUT it must be zero-filled anew.
+/* Bytes of workspace that sdattn_qk_stats, sdattn_softmax_av and sdattn_flash
+ * need for this shape on the current device (split-reduction partials plus
+ * arrival counters): enough for each of the three calls.  The same workspace
+ * serves all three calls and any shape whose need is at most its size.  It
+ * must be zero-filled once before its first use; every completed call leaves
+ * all of it zero again.  After SDATTN_ERR_TIMEOUT it must be zero-filled anew.
  * Returns 0 for an invalid descriptor. */
 size_t sdattn_workspace_bytes(const sdattn_desc *desc);
 
@@ -121,9 +122,20 @@ sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const f
 
 /* FlashAttention form: one kernel, tiled over keys with an online softmax,
  * A never stored.  Q, K, V: inputs; O: output.  LS_or_null: if not NULL,
- * also receives (L_i, S_i) as defined above. */
+ * also receives (L_i, S_i) as defined above.
+ * ws / ws_bytes: optional workspace (may be NULL / 0).  When given it must
+ * be zero-filled before first use and hold at least sdattn_workspace_bytes
+ * (desc) bytes (a short one returns SDATTN_ERR_WORKSPACE; the flash part of
+ * the need grows with the SM count and d, not with B, H, N or M); the kernel
+ * may then cut the key range
+ * of a block of query rows between two CTAs and merge the two halves'
+ * partial results (an online-softmax merge), which evens out the last wave
+ * of work when the row blocks do not divide evenly among the SMs.  Without
+ * it every block of rows runs whole in one CTA.  Results agree within
+ * rounding either way. */
 sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K,
-                           const void *V, void *O, float *LS_or_null, void *stream);
+                           const void *V, void *O, float *LS_or_null, void *ws,
+                           size_t ws_bytes, void *stream);
 
 /* Allocation-free variant of sdattn_qk_stats.  It has no counterpart in the
  * paper; it exists for callers that cannot allocate device memory (for

@@ -47,7 +47,7 @@ def test_a_ld_and_workspace(lib):
 def test_bad_descriptor(lib, kw, status):
     d = _desc(**kw)
     p = ctypes.c_void_p(4096)
-    assert lib.sdattn_flash(ctypes.byref(d), p, p, p, p, None, None) == status
+    assert lib.sdattn_flash(ctypes.byref(d), p, p, p, p, None, None, 0, None) == status
     assert lib.sdattn_qk_stats(ctypes.byref(d), p, p, p, p, p, 1 << 30, None) == status
     assert lib.sdattn_softmax_av(ctypes.byref(d), p, p, p, p, None, 0, None) == status
 
@@ -56,10 +56,10 @@ def test_null_and_misaligned_pointers(lib):
     d = _desc()
     ok = ctypes.c_void_p(1 << 20)
     bad = ctypes.c_void_p((1 << 20) + 8)
-    assert lib.sdattn_flash(None, ok, ok, ok, ok, None, None) == 1
-    assert lib.sdattn_flash(ctypes.byref(d), None, ok, ok, ok, None, None) == 1
-    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, bad, ok, None, None) == 3
-    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, bad, None) == 3
+    assert lib.sdattn_flash(None, ok, ok, ok, ok, None, None, 0, None) == 1
+    assert lib.sdattn_flash(ctypes.byref(d), None, ok, ok, ok, None, None, 0, None) == 1
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, bad, ok, None, None, 0, None) == 3
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, bad, None, 0, None) == 3
     assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, None, None, 0, None) == 1
     assert lib.sdattn_softmax_av(ctypes.byref(d), bad, ok, ok, ok, None, 0, None) == 3
     assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, bad, ok, 1 << 30, None) == 3
@@ -70,8 +70,14 @@ def test_workspace_checked(lib):
     ok = ctypes.c_void_p(1 << 20)
     need = lib.sdattn_workspace_bytes(ctypes.byref(d))
     assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, None, need, None) == 4
-    assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, ok, need - 1, None) == 4
+    assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, ok, 4096, None) == 4
     assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, ok, None, 16, None) == 4
+    # flash: the workspace is optional, but a size without a pointer, a short
+    # one or a misaligned one is refused before anything is enqueued
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, None, None, 16, None) == 4
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, None, ok, 4096, None) == 4
+    assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, None, bad, need, None) == 3
 
 
 def test_status_strings(lib):

@@ -29,7 +29,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert sd.device_error()[0] == "SDATTN_OK"
     os.environ["SDATTN_TEST_INJECT_STALL"] = "1"
     try:
-        sd.flash(tq, tk, tv)
+        sd.flash(tq, tk, tv, use_workspace=False)
         status, detail = sd.device_error()          # synchronises; about one second
     finally:
         del os.environ["SDATTN_TEST_INJECT_STALL"]

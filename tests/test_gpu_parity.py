@@ -174,6 +174,62 @@ def test_peaked_scores_rescale():
 
 
 # ---------------------------------------------------------------------------
+# flash with key ranges cut between CTAs
+# ---------------------------------------------------------------------------
+
+def _sms():
+    return torch.cuda.get_device_properties(DEV).multi_processor_count
+
+
+@pytest.mark.parametrize("N,M,d", [(200, 1000, 40), (100, 640, 80), (128, 300, 160)])
+def test_flash_split_key_ranges(N, M, d):
+    """SM count + 2 blocks of query rows: the last wave would be two blocks on
+    a nearly idle GPU, so with a workspace every CTA takes an equal share of
+    the (row block, key tile) pairs and the blocks cut between two CTAs are
+    merged.  Ragged rows and keys; both schedules against the oracle, the
+    split one twice (bitwise equal: the merge order is fixed), and the
+    workspace back at zero afterwards."""
+    H = _sms() + 2
+    rows_per_block = 256 if d == 40 else 128
+    N = min(N, rows_per_block)
+    shape = synth.Shape("split", 1, H, N, M, d)
+    q, k, v = synth.make_qkv(shape, 81, call_id=d)
+    scale = f32(1 / math.sqrt(d))
+    ref = oracle.attention(q, k, v, scale)
+    tq, tk, tv = to_dev(q, k, v)
+    desc = sd.make_desc(1, H, N, M, d, torch.float16, scale)
+    ws = torch.zeros(sd.workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    outs = []
+    for use_ws in (True, True, False):
+        obuf, o = guarded((1, H, N, d), tq.dtype)
+        lsbuf, ls = guarded((1, H, N, 2), torch.float32)
+        sd.flash(tq, tk, tv, scale, out=o, out_ls=ls, ws=ws if use_ws else None, use_workspace=use_ws)
+        torch.cuda.synchronize()
+        assert margins_intact(obuf) and margins_intact(lsbuf)
+        assert int(torch.count_nonzero(ws)) == 0
+        assert_o(o.float().cpu().numpy(), ref["O"], f"flash split={use_ws}")
+        ls_h = ls.cpu().numpy().astype(np.float64)
+        assert np.abs(ls_h[..., 0] - ref["L"]).max() <= L_TOL
+        assert np.abs(ls_h[..., 1] / ref["S"] - 1).max() <= S_RTOL_FLASH
+        outs.append((o.clone(), ls.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_flash_64x64_self_split_against_whole():
+    """The 64x64 self-attention (256 units of 2 x 128 rows on the SMs) with and
+    without the workspace: both within rounding of each other."""
+    shape = synth.CONFIGS[2]
+    q, k, v = synth.make_qkv(shape, 2)
+    tq, tk, tv = to_dev(q, k, v)
+    o1, ls1 = sd.flash(tq, tk, tv, return_ls=True)
+    o2, ls2 = sd.flash(tq, tk, tv, return_ls=True, use_workspace=False)
+    assert torch.equal(ls1[..., 0], ls2[..., 0])
+    assert torch.allclose(ls1[..., 1], ls2[..., 1], rtol=2 * S_RTOL_FLASH, atol=0)
+    ea, er = o_errors(o1.float().cpu().numpy(), o2.float().cpu().numpy().astype(np.float64))
+    assert ea <= 1e-3 and er <= 1e-3
+
+
+# ---------------------------------------------------------------------------
 # invariants on the GPU outputs
 # ---------------------------------------------------------------------------
 
