@@ -493,12 +493,17 @@ def choose_stride(budget_s: float) -> int:
 
 
 def cpu_baseline(seconds: float):
+    """The oracle on a row sample of the step set, repeated until about `seconds` of CPU work."""
     sample = OracleSample(choose_stride(seconds))
-    s = sample.run()
-    return {"value": round(sample.flops / s / 1e12, 6), "unit": "TFLOP/s", "cores": sample.oracle.max_threads(),
+    s, n = sample.run(), 1
+    while s < 0.8 * seconds and n < 16:
+        s += sample.run()
+        n += 1
+    return {"value": round(n * sample.flops / s / 1e12, 6), "unit": "TFLOP/s", "cores": sample.oracle.max_threads(),
             "kind": "oracle",
-            "sample": f"every {sample.stride}-th query row of all 32 calls of the step set "
-                      f"({sample.flops / 1e9:.2f} GFLOP of the {STEP_FLOPS / 1e9:.1f} GFLOP step), fp64 C + OpenMP",
+            "sample": f"{n} x every {sample.stride}-th query row of all 32 calls of the step set "
+                      f"({sample.flops / 1e9:.2f} GFLOP of the {STEP_FLOPS / 1e9:.1f} GFLOP step each time), "
+                      f"fp64 C + OpenMP",
             "seconds": round(s, 2)}
 
 
