@@ -145,6 +145,7 @@ struct FlashCfg {
   static constexpr int ROWF = (D + 3 + 3) / 4 * 4;
   static_assert(STAGES >= 2, "key/value ring too shallow");
   static_assert(NQ * QCOLS <= 512, "tensor memory budget");
+  static_assert(NQ >= 1 && NQ <= 3, "MMA warps 1..NQ share the first warp group with the TMA warp");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
   static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
@@ -173,12 +174,34 @@ __device__ __forceinline__ float4* partial_rows(float* part, int64_t slot, int h
   return reinterpret_cast<float4*>(part) + (slot * 2 + half) * (ROWF / 4) * 128;
 }
 
-// named barrier of query tile q's four softmax warps (ids fixed at compile time)
+// p = 2^(s*c - m) for one row's key tile, packed to 16-bit pairs: NPOLY of
+// every 8 pairs on the FMA pipe (exp2_poly2), the rest on MUFU.
+template <int BN, bool BF16, int NPOLY>
+__device__ __forceinline__ void flash_exp_block(const uint32_t (&v)[BN], uint64_t c2, uint64_t nm2,
+                                                uint32_t (&pk)[BN / 2]) {
+#pragma unroll
+  for (int k = 0; k < BN / 2; ++k) {
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), c2, nm2);
+    float x0, x1, e0, e1;
+    f2_unpack(x2, x0, x1);
+    if ((k & 7) < NPOLY) {
+      exp2_poly2(x0, x1, e0, e1);
+    } else {
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
+    }
+    pk[k] = pack2<BF16>(e0, e1);
+  }
+}
+
+// named barrier of query tile q's four softmax warps (ids 1 + q, fixed at compile time)
 __device__ __forceinline__ void softmax_bar_sync(int q) {
   if (q == 0)
     named_bar_sync(1, 128);
-  else
+  else if (q == 1)
     named_bar_sync(2, 128);
+  else
+    named_bar_sync(3, 128);
 }
 
 // One counter update for the tile: thread r == 0 adds v (acquire-release),
@@ -528,35 +551,21 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           for (int i = 0; i < w / 2; ++i) acc[i] = fmaxf(acc[i], acc[i + w / 2]);
         const float mx = acc[0];
         rawmax = fmaxf(rawmax, mx);
+        const float mt = mx * c;
+        const uint64_t c2 = f2_pack(c, c);
+        float alpha = 1.f;
+        bool rescale = false;
+        uint32_t pk[BN / 2];
         if (NQ == 2 && q == 0 && t == 0) {
           __syncwarp();
           if (lane == 0) mbar_arrive(stagger);
         }
-        const float mt = mx * c;
-        float alpha = 1.f;
-        bool rescale = false;
         if (mt > m_used + 8.f) {
           alpha = ex2_approx(m_used - mt);
           m_used = mt;
           rescale = (j > sg.j0);
         }
-        // p = 2^(s*c - m): NPOLY of every 8 pairs on the FMA pipe, the rest on MUFU
-        const uint64_t c2 = f2_pack(c, c);
-        const uint64_t nm2 = f2_pack(-m_used, -m_used);
-        uint32_t pk[BN / 2];
-#pragma unroll
-        for (int k = 0; k < BN / 2; ++k) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), c2, nm2);
-          float x0, x1, e0, e1;
-          f2_unpack(x2, x0, x1);
-          if ((k & 7) < NPOLY) {
-            exp2_poly2(x0, x1, e0, e1);
-          } else {
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          }
-          pk[k] = pack2<BF16>(e0, e1);
-        }
+        flash_exp_block<BN, BF16, NPOLY>(v, c2, f2_pack(-m_used, -m_used), pk);
         if (j > sg.j0) {
           // P V of the previous tile must be done: P is reused and O may be rescaled
           live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
