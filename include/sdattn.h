@@ -113,9 +113,9 @@ sdattn_status sdattn_qk_stats(const sdattn_desc *desc, const void *Q, const void
  * multiplication by V.
  *   O[b][h][i][c] = (sum_j exp(A_ij - L_i) V[b][h][j][c]) / S_i
  * A, LS (as written by sdattn_qk_stats), V: inputs; O: output.
- * ws / ws_bytes: optional workspace (may be NULL / 0); when given (at least
- * sdattn_workspace_bytes(desc) bytes, zero-filled before first use) the key
- * range may be split across CTAs for small problems. */
+ * ws / ws_bytes: optional workspace (may be NULL / 0), reserved: this
+ * version never splits a row's key range here and leaves a given workspace
+ * untouched (a size without a pointer is still refused). */
 sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const float *LS,
                                 const void *V, void *O, void *ws, size_t ws_bytes,
                                 void *stream);
