@@ -55,7 +55,7 @@ def parse_args():
     ap.add_argument("--no-side", action="store_true",
                     help="time the step set only (no per-form, per-kernel or end-to-end extras)")
     ap.add_argument("--case", default=None,
-                    help="FORM:CONFIG, e.g. flash:2 -- run one form on one configuration (for profilers)")
+                    help="FORM:WORKLOAD, e.g. flash:self64 -- run one form on one workload (for profilers)")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -330,7 +330,7 @@ def run_gpu(args, rank, world, local_rank):
 
     peaks, peak_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    dom_flops = synth.CONFIGS[2].flops
+    dom_flops = synth.WORKLOADS["self64"].flops
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     traffic = profiled_traffic()
     line = {
@@ -405,7 +405,7 @@ def side_measurements(torch, sd, stream, sets, scratch, issue, K):
 
     # headline kernels on the 64x64 self-attention (5 distinct calls per replay)
     dom = [i for i, c in enumerate(CALLS) if is_dominant(c)]
-    c2 = synth.CONFIGS[2]
+    c2 = synth.WORKLOADS["self64"]
     peaks, _ = measured_peaks()
     f_ms = time_graph(lambda s: issue(s, dom, lambda c: "flash"), K, len(dom))
     p_ms = time_graph(lambda s: issue(s, dom, lambda c: "partial"), max(K // 4, 5), len(dom))
@@ -573,14 +573,14 @@ def run_reference(args, rank, world):
 
 
 def run_case(args):
-    """One form on one configuration, `reps` launches after one warm-up, each
+    """One form on one named workload, `reps` launches after one warm-up, each
     timed with CUDA events; used as the target of profiler captures."""
     import torch
     import diffusion_unet_attention_b200 as sd
-    form, cid = args.case.split(":")
-    call = synth.CONFIGS[int(cid)]
+    form, name = args.case.split(":")
+    call = synth.WORKLOADS[name]
     device = torch.device("cuda", 0)
-    q, k, v = synth.make_qkv(call, int(cid))
+    q, k, v = synth.make_qkv(call, synth.STREAM[name])
     tq, tk, tv = (torch.from_numpy(x).to(device) for x in (q, k, v))
     o = torch.empty_like(tq)
     scratch = Scratch(sd, torch, device, [call])

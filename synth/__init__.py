@@ -88,16 +88,17 @@ class Shape:
         return 4 * self.B * self.H * self.N * self.M
 
 
-# Configurations of the benchmark study (id -> shape).  Seeds follow
-# 1000 * config_id + {Q: 0, K: 1, V: 2} + 10 * call_id.
-CONFIGS = {
-    1: Shape("tiny self-attention", 1, 1, 256, 256, 40),
-    2: Shape("64x64-latent self-attention", 2, 8, 4096, 4096, 40),
-    3: Shape("64x64-latent cross-attention", 2, 8, 4096, 77, 40),
-    4: Shape("32x32-latent self-attention", 2, 8, 1024, 1024, 80),
-    5: Shape("16x16-latent self-attention", 2, 8, 256, 256, 160),
-    6: Shape("8x8 mid-block self-attention", 2, 8, 64, 64, 160),
+# The single-call workloads of the study, by name, and the seed stream each
+# draws its inputs from.  Seeds follow 1000 * stream + {Q: 0, K: 1, V: 2} + 10 * call_id.
+WORKLOADS = {
+    "tiny": Shape("tiny self-attention", 1, 1, 256, 256, 40),
+    "self64": Shape("64x64-latent self-attention", 2, 8, 4096, 4096, 40),
+    "cross64": Shape("64x64-latent cross-attention", 2, 8, 4096, 77, 40),
+    "self32": Shape("32x32-latent self-attention", 2, 8, 1024, 1024, 80),
+    "self16": Shape("16x16-latent self-attention", 2, 8, 256, 256, 160),
+    "self8": Shape("8x8 mid-block self-attention", 2, 8, 64, 64, 160),
 }
+STREAM = {"tiny": 1, "self64": 2, "cross64": 3, "self32": 4, "self16": 5, "self8": 6}
 STEP_SET_ID = 7
 TEXT_TOKENS = 77
 
@@ -121,15 +122,15 @@ def unet_step_set(B: int = 2, H: int = 8):
     return calls
 
 
-def seeds(config_id: int, call_id: int = 0):
-    """(seed_Q, seed_K, seed_V) for one call of one configuration."""
-    base = 1000 * config_id + 10 * call_id
+def seeds(stream: int, call_id: int = 0):
+    """(seed_Q, seed_K, seed_V) for one call drawn from one seed stream."""
+    base = 1000 * stream + 10 * call_id
     return base + 0, base + 1, base + 2
 
 
-def make_qkv(shape: Shape, config_id: int, call_id: int = 0, dtype=np.float16):
+def make_qkv(shape: Shape, stream: int, call_id: int = 0, dtype=np.float16):
     """Seeded Q [B,H,N,d], K and V [B,H,M,d], N(0,1) rounded to `dtype`."""
-    sq, sk, sv = seeds(config_id, call_id)
+    sq, sk, sv = seeds(stream, call_id)
     q = normal(sq, (shape.B, shape.H, shape.N, shape.d), dtype)
     k = normal(sk, (shape.B, shape.H, shape.M, shape.d), dtype)
     v = normal(sv, (shape.B, shape.H, shape.M, shape.d), dtype)

@@ -110,8 +110,8 @@ def run_paths(q, k, v, scale, rows=None, check_a=True):
 def test_tiny_config_fp32_inputs_rounded():
     """Tiny config: fp32 N(0,1) inputs, rounded to fp16 (nearest even) on the
     device; the gated oracle runs on the rounded values."""
-    shape = synth.CONFIGS[1]
-    q32, k32, v32 = synth.make_qkv(shape, 1, dtype=np.float32)
+    shape = synth.WORKLOADS["tiny"]
+    q32, k32, v32 = synth.make_qkv(shape, synth.STREAM["tiny"], dtype=np.float32)
     tq, tk, tv = (t.half() for t in to_dev(q32, k32, v32))
     q, k, v = (t.cpu().numpy() for t in (tq, tk, tv))
     assert np.array_equal(q, q32.astype(np.float16))
@@ -124,22 +124,22 @@ def test_tiny_config_fp32_inputs_rounded():
     print(f"tiny config vs fp32-input oracle: max_abs {ea:.3e} rel_frob {er:.3e}")
 
 
-@pytest.mark.parametrize("cid", [3, 4, 5, 6])
-def test_config_full(cid):
-    shape = synth.CONFIGS[cid]
-    q, k, v = synth.make_qkv(shape, cid)
+@pytest.mark.parametrize("name", ["cross64", "self32", "self16", "self8"])
+def test_workload_full(name):
+    shape = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(shape, synth.STREAM[name])
     scale = f32(1 / math.sqrt(shape.d))
     rows = None if shape.N <= 1024 else np.arange(0, shape.N, 3)
     res, _ = run_paths(q, k, v, scale, rows=rows, check_a=shape.M <= 1024)
-    print(cid, res)
+    print(name, res)
 
 
-def test_config_64x64_self_sampled():
+def test_workload_64x64_self_sampled():
     """64x64-latent self-attention at full size (B=2, H=8, N=M=4096, d=40) in the
     launch configuration the benchmark times; the oracle computes a sample of
     query rows (every tile and the first and last rows of each)."""
-    shape = synth.CONFIGS[2]
-    q, k, v = synth.make_qkv(shape, 2)
+    shape = synth.WORKLOADS["self64"]
+    q, k, v = synth.make_qkv(shape, synth.STREAM["self64"])
     scale = f32(1 / math.sqrt(40))
     rows = np.unique(np.concatenate([np.arange(0, 4096, 61), np.arange(127, 4096, 128), [4095]]))
     res, _ = run_paths(q, k, v, scale, rows=rows, check_a=True)
@@ -218,8 +218,8 @@ def test_flash_split_key_ranges(N, M, d):
 def test_flash_64x64_self_split_against_whole():
     """The 64x64 self-attention (256 units of 2 x 128 rows on the SMs) with and
     without the workspace: both within rounding of each other."""
-    shape = synth.CONFIGS[2]
-    q, k, v = synth.make_qkv(shape, 2)
+    shape = synth.WORKLOADS["self64"]
+    q, k, v = synth.make_qkv(shape, synth.STREAM["self64"])
     tq, tk, tv = to_dev(q, k, v)
     o1, ls1 = sd.flash(tq, tk, tv, return_ls=True)
     o2, ls2 = sd.flash(tq, tk, tv, return_ls=True, use_workspace=False)

@@ -39,7 +39,7 @@ def test_step_set_shapes():
 
 def test_seeds_distinct_per_tensor_and_call():
     s = set()
-    for cid in range(1, 8):
+    for stream in range(1, 8):
         for call in range(32):
-            s.update(synth.seeds(cid, call))
+            s.update(synth.seeds(stream, call))
     assert len(s) == 7 * 32 * 3
