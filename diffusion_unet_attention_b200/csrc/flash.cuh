@@ -518,8 +518,12 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         if (!live) break;
         tc_fence_after();
         uint32_t v[BN];
+        if constexpr (BN == 128) {
+          tmem_ld_x128(s_tmem, v);
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_x32(s_tmem + cc * 32, v + cc * 32);
+          for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_x32(s_tmem + cc * 32, v + cc * 32);
+        }
         tmem_wait_ld();
         reg_fence<BN>(v);
         tc_fence_before();
@@ -585,8 +589,12 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
             }
           }
         }
+        if constexpr (BN == 128) {
+          tmem_st_x64(p_tmem, pk);
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) tmem_st_x16(p_tmem + cc * 16, pk + cc * 16);
+          for (int cc = 0; cc < BN / 32; ++cc) tmem_st_x16(p_tmem + cc * 16, pk + cc * 16);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

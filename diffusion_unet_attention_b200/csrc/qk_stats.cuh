@@ -234,8 +234,7 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
         if (!live) break;
         tc_fence_after();
         uint32_t v[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_x32(tmem + ab * 128 + c * 32 + lane_off, v + 32 * c);
+        tmem_ld_x128(tmem + ab * 128 + lane_off, v);
         tmem_wait_ld();
         reg_fence<128>(v);
         tc_fence_before();
