@@ -605,28 +605,24 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
       if (!live) break;
       tc_fence_after();
-      float l;
-      {
-        uint32_t o[8];
-        tmem_ld_x8(o_tmem + D, o);
-        tmem_wait_ld();
-        reg_fence<8>(o);
-        l = __uint_as_float(o[0]);
-      }
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row) * D * 2;
       if (!(p.split && sg.cut(p))) {
+        // O's D columns and the row sum l (column D), one tensor-memory wait
+        uint32_t o[D + 8];
+#pragma unroll
+        for (int c8 = 0; c8 <= D / 8; ++c8) tmem_ld_x8(o_tmem + c8 * 8, o + c8 * 8);
+        tmem_wait_ld();
+        reg_fence<D + 8>(o);
+        const float l = __uint_as_float(o[D]);
         const float inv = 1.f / l;
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
-          uint32_t o[8];
-          tmem_ld_x8(o_tmem + c8 * 8, o);
-          tmem_wait_ld();
-          reg_fence<8>(o);
+          const uint32_t* oc = o + c8 * 8;
           uint4 w;
-          w.x = pack2<BF16>(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
-          w.y = pack2<BF16>(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
-          w.z = pack2<BF16>(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
-          w.w = pack2<BF16>(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+          w.x = pack2<BF16>(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+          w.y = pack2<BF16>(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+          w.z = pack2<BF16>(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+          w.w = pack2<BF16>(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
           if (row < p.N) *reinterpret_cast<uint4*>(orow + c8 * 16) = w;
         }
         if (p.LS != nullptr && row < p.N) {
@@ -635,6 +631,14 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(L, S);
         }
       } else if (kcut < 2) {
+        float l;
+        {
+          uint32_t o[8];
+          tmem_ld_x8(o_tmem + D, o);
+          tmem_wait_ld();
+          reg_fence<8>(o);
+          l = __uint_as_float(o[0]);
+        }
         const int side = sg.j0 > 0 ? 1 : 0;   // 0: head half, 1: tail half
         flash_cut_epilogue<D, BF16, C::ROWF>(p.part, p.tickets, p.LS, p.N, p.scale, c, o_tmem, side,
                                             static_cast<int64_t>(blockIdx.x - side) * NQ + q, q, r, bh, row, m_used,
