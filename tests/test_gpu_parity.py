@@ -215,6 +215,24 @@ def test_flash_split_key_ranges(N, M, d):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+def test_flash_split_bf16_reported():
+    """The key-range split with bf16 inputs, against the looser bf16 bound."""
+    H = _sms() + 2
+    shape = synth.Shape("split bf16", 1, H, 256, 1000, 40)
+    q, k, v = synth.make_qkv(shape, 82, dtype=np.float32)
+    tq, tk, tv = (t.bfloat16() for t in to_dev(q, k, v))
+    qb, kb, vb = (t.float().cpu().numpy() for t in (tq, tk, tv))
+    ref = oracle.attention(qb, kb, vb, f32(1 / math.sqrt(40)))
+    desc = sd.make_desc(1, H, 256, 1000, 40, torch.bfloat16, f32(1 / math.sqrt(40)))
+    ws = torch.zeros(sd.workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    o = sd.flash(tq, tk, tv, ws=ws)
+    torch.cuda.synchronize()
+    assert int(torch.count_nonzero(ws)) == 0
+    ea, er = o_errors(o.float().cpu().numpy(), ref["O"])
+    print(f"bf16 flash split: max_abs {ea:.3e} rel_frob {er:.3e}")
+    assert ea <= 2e-2 and er <= 8e-3
+
+
 def test_flash_64x64_self_split_against_whole():
     """The 64x64 self-attention (256 units of 2 x 128 rows on the SMs) with and
     without the workspace: both within rounding of each other."""
