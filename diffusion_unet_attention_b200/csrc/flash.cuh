@@ -9,13 +9,14 @@
 //
 // B200 design.  One persistent CTA per SM walks (b*H + h, group of NQ
 // 128-row query tiles) units, whole, or, when the units do not fill the last
-// wave, as equal shares of all (unit, key tile) pairs, a unit cut between two
-// CTAs being merged by the one that finishes second.  Roles:
+// wave, as equal shares of all (unit, key tile) pairs; a unit cut between two
+// CTAs is merged by one of its halves (flash_cut_epilogue).  Roles:
 //   warp 0            TMA producer: the unit's NQ Q tiles, then a ring of
 //                     (K tile, V tile) stages, 128-byte swizzled, no multicast;
-//   warp 1            tcgen05 MMA issuer: S = Q K^T into tensor memory; once
-//                     the softmax has written P (16-bit, aliasing S in tensor
-//                     memory) O += P V with O accumulated in tensor memory;
+//   warp 1 + q        tcgen05 MMA issuer for query tile q: S = Q K^T into
+//                     tensor memory; once the softmax has written P (16-bit,
+//                     its own tensor-memory buffer) O += P V, with O
+//                     accumulated in tensor memory;
 //   warps 4+4q..7+4q  softmax for query tile q, one row per thread: row max,
 //                     p = 2^(s*scale*log2e - m), row sum, P packed to 16 bits,
 //                     and the rescale of O when the running max grows.
