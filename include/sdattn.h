@@ -125,14 +125,14 @@ sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const f
  * also receives (L_i, S_i) as defined above.
  * ws / ws_bytes: optional workspace (may be NULL / 0).  When given it must
  * be zero-filled before first use and hold at least sdattn_workspace_bytes
- * (desc) bytes (a short one returns SDATTN_ERR_WORKSPACE; the flash part of
- * the need grows with the SM count and d, not with B, H, N or M); the kernel
- * may then cut the key range
- * of a block of query rows between two CTAs and merge the two halves'
- * partial results (an online-softmax merge), which evens out the last wave
- * of work when the row blocks do not divide evenly among the SMs.  Without
- * it every block of rows runs whole in one CTA.  Results agree within
- * rounding either way. */
+ * (desc) bytes; a short one returns SDATTN_ERR_WORKSPACE.  The flash part of
+ * that need grows with the SM count and d, not with B, H, N or M.  With a
+ * workspace the kernel may cut the key range of a block of query rows
+ * between two CTAs and merge the two halves' partial results (an
+ * online-softmax merge, in a fixed order, so repeated calls give identical
+ * results); this evens out the last wave of work when the row blocks do not
+ * divide evenly among the SMs.  Without it every block of rows runs whole in
+ * one CTA.  The two schedules agree within rounding. */
 sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K,
                            const void *V, void *O, float *LS_or_null, void *ws,
                            size_t ws_bytes, void *stream);
