@@ -25,7 +25,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -39,8 +38,15 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-FLASH_SRC = ("diffusion_unet_attention_b200/csrc/flash.cuh", "diffusion_unet_attention_b200/csrc/sm100.cuh")
-PROFILE_MD = os.path.join(ROOT, "profiles", "flash_64x64_self_d40.md")
+# Sources each profiled kernel is built from; a committed ncu summary
+# (profiles/<name>.json) counts only while its recorded digest matches them.
+CSRC = "diffusion_unet_attention_b200/csrc/"
+KERNEL_SRC = {
+    "flash": (CSRC + "flash.cuh", CSRC + "sm100.cuh", CSRC + "sdattn.cu"),
+    "qk_stats": (CSRC + "qk_stats.cuh", CSRC + "sm100.cuh", CSRC + "sdattn.cu"),
+    "softmax_av": (CSRC + "softmax_av.cuh", CSRC + "sm100.cuh", CSRC + "sdattn.cu"),
+}
+PROFILE_JSON = {k: os.path.join(ROOT, "profiles", f"{k}_64x64_self_d40.json") for k in KERNEL_SRC}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -69,6 +75,17 @@ WORKLOAD = ("SD1.4 512x512 UNet step attention set: 16 transformer blocks x (sel
             "B=2, H=8, d=40/80/160, fp16 N(0,1); flash for d=40, partially fused softmax otherwise")
 
 
+# bytes of one input set (Q, K, V of every call, fp16)
+SET_BYTES = sum(2 * c.B * c.H * (c.N + 2 * c.M) * c.d for c in CALLS)
+
+
+def job_config(world: int) -> dict:
+    """The `config` of the JSON line, the same for both arms."""
+    return {"workload": WORKLOAD, "calls_per_step": len(CALLS), "flops_per_step": STEP_FLOPS,
+            "accumulate": "f32", "l2": "two input sets of %.0f MB alternate (each > 126 MB L2)" % (SET_BYTES / 1e6),
+            "timing": "CUDA graph replay per step, CUDA events", "parallelism": f"replicas x{world}"}
+
+
 def policy_form(call) -> str:
     return "flash" if call.d == 40 else "partial"
 
@@ -87,25 +104,35 @@ def measured_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_digest() -> str:
+def source_digest(kernel: str = "flash") -> str:
+    """First 16 hex digits of the SHA-256 over the kernel's source files."""
     h = hashlib.sha256()
-    for rel in FLASH_SRC:
+    for rel in KERNEL_SRC[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """Per-launch DRAM bytes of the flash kernel on the 64x64 self-attention,
-    from the committed ncu summary, if it was taken on the current source."""
+def profiled(kernel: str = "flash"):
+    """The committed ncu figures of `kernel` on the 64x64 self-attention
+    (profiles/<kernel>_64x64_self_d40.json), or None when they are missing or
+    were taken on other sources than the current ones."""
     try:
-        text = open(PROFILE_MD).read()
-    except OSError:
+        with open(PROFILE_JSON[kernel]) as f:
+            prof = json.load(f)
+    except (OSError, ValueError):
         return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s*\(source\s+([0-9a-f]+)\)", text)
-    if not m or m.group(2) != source_digest():
+    if prof.get("source_digest") != source_digest(kernel):
         return None
-    return float(m.group(1))
+    return prof
+
+
+def profiled_traffic(kernel: str = "flash"):
+    """Per-launch DRAM bytes (read + write) of `kernel` from its current profile."""
+    prof = profiled(kernel)
+    if prof is None:
+        return None
+    return float(prof["dram_bytes_read"] + prof["dram_bytes_write"])
 
 
 # ----------------------------------------------------------------------------
@@ -194,6 +221,7 @@ class StepSet:
     def __init__(self, sd, torch, device, set_id: int):
         self.sd, self.torch, self.device = sd, torch, device
         self.inputs = []
+        self.device = device
         for ci, call in enumerate(CALLS):
             q, k, v = synth.make_qkv(call, synth.STEP_SET_ID + 10 * set_id, call_id=ci)
             tq, tk, tv = (torch.from_numpy(x).to(device) for x in (q, k, v))
@@ -219,15 +247,20 @@ class Scratch:
         ws = max(sd.workspace_bytes(sd.make_desc(c.B, c.H, c.N, c.M, c.d, torch.float16, 1.0)) for c in calls)
         self.ws = torch.zeros(max(ws, 256), dtype=torch.uint8, device=device)
 
+    def views(self, call):
+        """A [B,H,N,lda] and LS [B,H,N,2] views of the shared scratch for `call`."""
+        lda = (call.M + 3) // 4 * 4
+        a = self.a[:call.B * call.H * call.N * lda].view(call.B, call.H, call.N, lda)
+        ls = self.ls[:call.B * call.H * call.N * 2].view(call.B, call.H, call.N, 2)
+        return a, ls
+
     def run(self, call, q, k, v, o, form):
         sd = self.sd
         scale = 1.0 / math.sqrt(call.d)
         if form == "flash":
             sd.flash(q, k, v, scale, out=o, ws=self.ws)
             return 1
-        lda = (call.M + 3) // 4 * 4
-        a = self.a[:call.B * call.H * call.N * lda].view(call.B, call.H, call.N, lda)
-        ls = self.ls[:call.B * call.H * call.N * 2].view(call.B, call.H, call.N, 2)
+        a, ls = self.views(call)
         sd.qk_stats(q, k, scale, out_a=a, out_ls=ls, ws=self.ws)
         sd.softmax_av(a, ls, v, scale, out=o)
         return 2
@@ -320,6 +353,7 @@ def run_gpu(args, rank, world, local_rank):
     e2e = None
     if rank == 0 and not args.no_side:
         extra = side_measurements(torch, sd, stream, sets, scratch, issue, K=min(K, 50))
+        extra["per_call"] = per_call_table(torch, sd, stream, sets[0], scratch)
     if not args.no_side:
         # every rank feeds its own replica from host memory; the job's step is its slowest rank's
         barrier()
@@ -346,10 +380,7 @@ def run_gpu(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f16",
         "data": "synthetic N(0,1), seeded SplitMix64/Box-Muller, fp16",
-        "config": {"workload": WORKLOAD, "calls_per_step": len(CALLS), "flops_per_step": STEP_FLOPS,
-                   "accumulate": "f32", "l2": "two input sets of %.0f MB alternate (each > 126 MB L2)"
-                   % (sets[0].h2d_bytes() / 1e6), "timing": "CUDA graph replay per step, CUDA events",
-                   "parallelism": f"replicas x{world}"},
+        "config": job_config(world),
         "gpu_launches": launches_per_step * K,
         "roofline": {"bound": "tensor", "kernel": "flash_kernel<40,2,128> on 64x64 self-attention",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
@@ -419,6 +450,68 @@ def side_measurements(torch, sd, stream, sets, scratch, issue, K):
                             "frac_measured_hbm": round(pf_bytes / (p_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
     }
     return out
+
+
+def per_call_table(torch, sd, stream, stepset, scratch, reps=15):
+    """Every distinct call of the step set in both forms, each timed alone with
+    CUDA events after an L2 flush (a 256 MB write), median of `reps`.  Rows
+    carry the call's algorithmic FLOPs and bytes, its fraction of the measured
+    tensor (flash) or HBM (partially fused) peak, and its time over its floor:
+    the larger of the FLOP floor, the byte floor and the measured time of a
+    minimal kernel launch timed the same way."""
+    peaks, _ = measured_peaks()
+    tflops_peak, hbm = float(peaks["bf16_tflops"]), float(peaks["hbm_gbs"])
+    dev = stepset.device
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    tiny = torch.empty(4, dtype=torch.float32, device=dev)
+    seen = {}
+    for i, c in enumerate(CALLS):
+        seen.setdefault((c.N, c.M, c.d), []).append(i)
+
+    def median_ms(fns):
+        """Per function in `fns` (issued back to back), the median time in ms."""
+        ts = [[] for _ in fns]
+        with torch.cuda.stream(stream):
+            for _ in range(reps + 2):
+                flush.zero_()
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+                ev[0].record(stream)
+                for j, fn in enumerate(fns):
+                    fn()
+                    ev[j + 1].record(stream)
+                stream.synchronize()
+                for j in range(len(fns)):
+                    ts[j].append(ev[j].elapsed_time(ev[j + 1]))
+        return [statistics.median(t[2:]) for t in ts]
+
+    launch_ms = median_ms([lambda: tiny.zero_()])[0]
+    rows = []
+    for (N, M, d), idxs in seen.items():
+        call, q, k, v, o = stepset.inputs[idxs[0]]
+        scale = 1.0 / math.sqrt(d)
+        a, ls = scratch.views(call)
+        f_ms, = median_ms([lambda: sd.flash(q, k, v, scale, out=o, ws=scratch.ws)])
+        qk_ms, av_ms = median_ms([lambda: sd.qk_stats(q, k, scale, out_a=a, out_ls=ls, ws=scratch.ws),
+                                  lambda: sd.softmax_av(a, ls, v, scale, out=o)])
+        io = 2 * call.B * call.H * (2 * call.N + 2 * call.M) * d          # Q, K, V read, O written
+        pf_bytes = io + 2 * call.a_bytes() + 2 * 8 * call.B * call.H * call.N   # + A written, read; LS
+        p_ms = qk_ms + av_ms
+        fl_floor = max(call.flops / (tflops_peak * 1e9), io / (hbm * 1e6), launch_ms)
+        pf_floor = max(call.flops / (tflops_peak * 1e9), pf_bytes / (hbm * 1e6), 2 * launch_ms)
+        rows.append({
+            "call": call.name.split(" ", 1)[1], "N": N, "M": M, "d": d, "per_step": len(idxs),
+            "policy": policy_form(call), "gflop": round(call.flops / 1e9, 3),
+            "flash": {"us": round(f_ms * 1e3, 2), "tflops": round(call.flops / (f_ms * 1e-3) / 1e12, 1),
+                      "frac_tensor": round(call.flops / (f_ms * 1e-3) / 1e12 / tflops_peak, 4),
+                      "x_floor": round(f_ms / fl_floor, 2)},
+            "partial": {"us": round(p_ms * 1e3, 2), "qk_stats_us": round(qk_ms * 1e3, 2),
+                        "softmax_av_us": round(av_ms * 1e3, 2), "mb": round(pf_bytes / 1e6, 2),
+                        "gbs": round(pf_bytes / (p_ms * 1e-3) / 1e9, 1),
+                        "frac_hbm": round(pf_bytes / (p_ms * 1e-3) / 1e9 / hbm, 4),
+                        "x_floor": round(p_ms / pf_floor, 2)},
+        })
+    return {"launch_floor_us": round(launch_ms * 1e3, 2), "note": "each call alone after an L2 flush; "
+            "x_floor = time / max(FLOP floor, byte floor, minimal launch)", "rows": rows}
 
 
 def end_to_end(torch, sd, stream, stepset, scratch, steps):
@@ -550,12 +643,25 @@ def cpu_baseline(seconds: float):
             "seconds": round(s, 2)}
 
 
+def reference_stride(steps_total: int, budget_s: float = 150.0) -> int:
+    """Row stride of each reference step: 1 (the whole step set) when
+    `steps_total` whole steps fit in about `budget_s` seconds of oracle time,
+    else the smallest stride whose sampled steps do."""
+    probe = OracleSample(256)
+    rate = probe.flops / max(probe.run(), 1e-6)
+    full_s = STEP_FLOPS / rate
+    return max(1, math.ceil(full_s * steps_total / budget_s))
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle, as it stands, on the host cores,
+    K timed steps after W untimed ones, each step the whole 32-call set when
+    the run fits in a few minutes (else the same row sample of every call).
+    `ms_per_step` is the measured time of one of those steps."""
     if rank != 0:
         return
     K, W = args.steps, args.warmup
-    budget = 90.0 / max(K + W, 1)          # whole run about a minute and a half
-    sample = OracleSample(choose_stride(budget))
+    sample = OracleSample(reference_stride(K + W))
     for _ in range(W):
         sample.run()
     tot_s = 0.0
@@ -563,14 +669,17 @@ def run_reference(args, rank, world):
         tot_s += sample.run()
     value = sample.flops * K / tot_s / 1e12
     thr = sample.oracle.max_threads()
+    what = ("the whole step set (all query rows of all 32 calls)" if sample.stride == 1 else
+            f"every {sample.stride}-th query row of all 32 calls ({sample.flops / 1e9:.3f} of "
+            f"{STEP_FLOPS / 1e9:.1f} GFLOP)")
     line = {"metric": "attention us & TFLOP/s per UNet-step set (1xB200); % of tensor / HBM roofline",
             "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": round(STEP_FLOPS / (value * 1e12) * 1e3, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD}, "impl": "reference",
+            "ms_per_step": round(tot_s / K * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic N(0,1), seeded SplitMix64/Box-Muller, fp16 widened to fp64",
+            "config": job_config(world), "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                             "sample": f"every {sample.stride}-th query row of all 32 calls per step "
-                                       f"({sample.flops / 1e9:.3f} GFLOP per step)"},
+                             "sample": f"each step: {what}, fp64 C + OpenMP", "seconds": round(tot_s, 2)},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -588,9 +697,7 @@ def run_case(args):
     o = torch.empty_like(tq)
     scratch = Scratch(sd, torch, device, [call])
     scale = 1.0 / math.sqrt(call.d)
-    lda = (call.M + 3) // 4 * 4
-    a = scratch.a[:call.B * call.H * call.N * lda].view(call.B, call.H, call.N, lda)
-    ls = scratch.ls[:call.B * call.H * call.N * 2].view(call.B, call.H, call.N, 2)
+    a, ls = scratch.views(call)
 
     def once():
         if form == "flash":

@@ -11,6 +11,10 @@ three optimisations, attention-efficiency paragraphs):
   `softmax_av` fuses the normalisation with the product by V;
 * FlashAttention: `flash` tiles over keys with an online softmax in one kernel.
 
+Variants of the partially fused form: the page's reduction as a kernel of its
+own over a stored A (`qk_scores`, `row_stats`, then `softmax_av`), and A
+stored in fp16 (`qk_stats_f16a`, `softmax_av_f16a`).
+
 This module only marshals torch tensors (device memory and streams) into the
 C ABI of libsdattn.so; all arithmetic runs in the CUDA kernels.  There is no
 CPU fallback: calls fail if the library or a CUDA device is missing.
@@ -24,8 +28,8 @@ import torch
 
 from . import _lib
 
-__all__ = ["qk_stats", "softmax_av", "flash", "partially_fused", "device_error", "a_ld", "workspace_bytes",
-           "SdattnError", "load_library"]
+__all__ = ["qk_stats", "softmax_av", "flash", "partially_fused", "qk_scores", "row_stats", "qk_stats_f16a",
+           "softmax_av_f16a", "device_error", "a_ld", "a16_ld", "workspace_bytes", "SdattnError", "load_library"]
 
 SdattnError = _lib.SdattnError
 load_library = _lib.load
@@ -73,6 +77,13 @@ def a_ld(desc: _lib.Desc) -> int:
     v = _lib_handle().sdattn_a_ld(ctypes.byref(desc))
     if v < 0:
         raise _lib.SdattnError("sdattn_a_ld", 1)
+    return int(v)
+
+
+def a16_ld(desc: _lib.Desc) -> int:
+    v = _lib_handle().sdattn_a16_ld(ctypes.byref(desc))
+    if v < 0:
+        raise _lib.SdattnError("sdattn_a16_ld", 1)
     return int(v)
 
 
@@ -135,8 +146,87 @@ def softmax_av(a: torch.Tensor, ls: torch.Tensor, v: torch.Tensor, scale: float 
     v = _contig(v)
     O = out if out is not None else torch.empty((B, H, N, d), dtype=v.dtype, device=v.device)
     st = _lib_handle().sdattn_softmax_av(ctypes.byref(desc), a.data_ptr(), ls.data_ptr(), v.data_ptr(),
-                                         O.data_ptr(), None, 0, _stream(v.device))
+                                         O.data_ptr(), _stream(v.device))
     _lib.check("sdattn_softmax_av", st)
+    return O
+
+
+def qk_scores(q: torch.Tensor, k: torch.Tensor, scale: float | None = None, out_a: torch.Tensor | None = None):
+    """Three-pass variant, first pass: A [B,H,N,lda] fp32 alone (no statistics)."""
+    B, H, N, M, d = _check_qk(q, k)
+    q, k = _contig(q), _contig(k)
+    desc = make_desc(B, H, N, M, d, q.dtype, _scale(scale, d))
+    lda = a_ld(desc)
+    A = out_a if out_a is not None else torch.empty((B, H, N, lda), dtype=torch.float32, device=q.device)
+    if A.shape != (B, H, N, lda) or A.dtype != torch.float32 or not A.is_contiguous():
+        raise ValueError(f"out_a must be contiguous fp32 [B,H,N,{lda}]")
+    st = _lib_handle().sdattn_qk_scores(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), A.data_ptr(),
+                                        _stream(q.device))
+    _lib.check("sdattn_qk_scores", st)
+    return A
+
+
+def row_stats(a: torch.Tensor, M: int, d: int, dtype: torch.dtype = torch.float16, out_ls: torch.Tensor | None = None,
+              ws: torch.Tensor | None = None):
+    """Three-pass variant, second pass: LS [B,H,N,2] = (L_i, S_i) of a stored
+    A [B,H,N,lda] (the stand-alone reduction kernel).  `M` is the number of
+    valid columns; `d` and `dtype` only complete the call's descriptor."""
+    if a.dim() != 4 or a.dtype != torch.float32 or not a.is_contiguous() or not a.is_cuda:
+        raise ValueError("a must be a contiguous fp32 CUDA tensor [B,H,N,lda]")
+    B, H, N, lda = a.shape
+    desc = make_desc(B, H, N, M, d, dtype, 1.0)
+    if lda != a_ld(desc):
+        raise ValueError(f"a's row stride {lda} does not match M={M}")
+    LS = out_ls if out_ls is not None else torch.empty((B, H, N, 2), dtype=torch.float32, device=a.device)
+    if LS.shape != (B, H, N, 2) or LS.dtype != torch.float32 or not LS.is_contiguous():
+        raise ValueError("out_ls must be contiguous fp32 [B,H,N,2]")
+    w = ws if ws is not None else workspace(desc, a.device)
+    st = _lib_handle().sdattn_row_stats(ctypes.byref(desc), a.data_ptr(), LS.data_ptr(), w.data_ptr(), w.numel(),
+                                        _stream(a.device))
+    _lib.check("sdattn_row_stats", st)
+    return LS
+
+
+def qk_stats_f16a(q: torch.Tensor, k: torch.Tensor, scale: float | None = None,
+                  out_a: torch.Tensor | None = None, out_ls: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None):
+    """fp16-A variant, first kernel: A16 [B,H,N,lda16] fp16 = fp16(scale Q K^T)
+    and LS [B,H,N,2], the statistics of the stored values."""
+    B, H, N, M, d = _check_qk(q, k)
+    q, k = _contig(q), _contig(k)
+    desc = make_desc(B, H, N, M, d, q.dtype, _scale(scale, d))
+    lda = a16_ld(desc)
+    A = out_a if out_a is not None else torch.empty((B, H, N, lda), dtype=torch.float16, device=q.device)
+    LS = out_ls if out_ls is not None else torch.empty((B, H, N, 2), dtype=torch.float32, device=q.device)
+    if A.shape != (B, H, N, lda) or A.dtype != torch.float16 or not A.is_contiguous():
+        raise ValueError(f"out_a must be contiguous fp16 [B,H,N,{lda}]")
+    if LS.shape != (B, H, N, 2) or LS.dtype != torch.float32 or not LS.is_contiguous():
+        raise ValueError("out_ls must be contiguous fp32 [B,H,N,2]")
+    w = ws if ws is not None else workspace(desc, q.device)
+    st = _lib_handle().sdattn_qk_stats_f16a(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), A.data_ptr(),
+                                            LS.data_ptr(), w.data_ptr(), w.numel(), _stream(q.device))
+    _lib.check("sdattn_qk_stats_f16a", st)
+    return A, LS
+
+
+def softmax_av_f16a(a: torch.Tensor, ls: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+                    out: torch.Tensor | None = None):
+    """fp16-A variant, second kernel: O from A16 and LS as written by `qk_stats_f16a`."""
+    B, H, M, d = v.shape
+    N = a.shape[2]
+    if not v.is_cuda:
+        raise ValueError("v must live on a CUDA device")
+    desc = make_desc(B, H, N, M, d, v.dtype, _scale(scale, d))
+    lda = a16_ld(desc)
+    if a.shape != (B, H, N, lda) or a.dtype != torch.float16 or not a.is_contiguous():
+        raise ValueError(f"a must be contiguous fp16 [B,H,N,{lda}]")
+    if ls.shape != (B, H, N, 2) or ls.dtype != torch.float32 or not ls.is_contiguous():
+        raise ValueError("ls must be contiguous fp32 [B,H,N,2]")
+    v = _contig(v)
+    O = out if out is not None else torch.empty((B, H, N, d), dtype=v.dtype, device=v.device)
+    st = _lib_handle().sdattn_softmax_av_f16a(ctypes.byref(desc), a.data_ptr(), ls.data_ptr(), v.data_ptr(),
+                                              O.data_ptr(), _stream(v.device))
+    _lib.check("sdattn_softmax_av_f16a", st)
     return O
 
 
@@ -168,10 +258,24 @@ def flash(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None
     return (O, LS) if (return_ls or out_ls is not None) else O
 
 
-def partially_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None):
-    """Both partially fused kernels back to back; returns O."""
-    A, LS = qk_stats(q, k, scale)
-    return softmax_av(A, LS, v, scale)
+def partially_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+                    variant: str = "fused"):
+    """The partially fused form; returns O.
+
+    variant "fused": qk_stats then softmax_av (statistics in the QK^T epilogue);
+    "three_pass": qk_scores, row_stats, softmax_av (the stand-alone reduction);
+    "f16a": qk_stats_f16a then softmax_av_f16a (A stored in fp16)."""
+    if variant == "fused":
+        A, LS = qk_stats(q, k, scale)
+        return softmax_av(A, LS, v, scale)
+    if variant == "three_pass":
+        A = qk_scores(q, k, scale)
+        LS = row_stats(A, k.shape[2], q.shape[3], q.dtype)
+        return softmax_av(A, LS, v, scale)
+    if variant == "f16a":
+        A, LS = qk_stats_f16a(q, k, scale)
+        return softmax_av_f16a(A, LS, v, scale)
+    raise ValueError(f"unknown variant {variant!r}")
 
 
 def device_error():

@@ -27,7 +27,9 @@ STATUS = {
 
 # Every symbol include/sdattn.h declares.
 EXPORTS = ("sdattn_a_ld", "sdattn_workspace_bytes", "sdattn_qk_stats", "sdattn_softmax_av", "sdattn_flash",
-           "sdattn_qk_stats_noalloc", "sdattn_device_error", "sdattn_status_string", "sdattn_version")
+           "sdattn_qk_scores", "sdattn_row_stats", "sdattn_a16_ld", "sdattn_qk_stats_f16a",
+           "sdattn_softmax_av_f16a", "sdattn_qk_stats_noalloc", "sdattn_device_error", "sdattn_status_string",
+           "sdattn_version")
 
 
 class Desc(ctypes.Structure):
@@ -62,8 +64,18 @@ def load(path: str = LIB_PATH):
     lib.sdattn_workspace_bytes.restype = sz
     lib.sdattn_qk_stats.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
     lib.sdattn_qk_stats.restype = ctypes.c_int
-    lib.sdattn_softmax_av.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sdattn_softmax_av.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.sdattn_softmax_av.restype = ctypes.c_int
+    lib.sdattn_qk_scores.argtypes = [dp, vp, vp, vp, vp]
+    lib.sdattn_qk_scores.restype = ctypes.c_int
+    lib.sdattn_row_stats.argtypes = [dp, vp, vp, vp, sz, vp]
+    lib.sdattn_row_stats.restype = ctypes.c_int
+    lib.sdattn_a16_ld.argtypes = [dp]
+    lib.sdattn_a16_ld.restype = ctypes.c_int64
+    lib.sdattn_qk_stats_f16a.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sdattn_qk_stats_f16a.restype = ctypes.c_int
+    lib.sdattn_softmax_av_f16a.argtypes = [dp, vp, vp, vp, vp, vp]
+    lib.sdattn_softmax_av_f16a.restype = ctypes.c_int
     lib.sdattn_flash.argtypes = [dp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.sdattn_flash.restype = ctypes.c_int
     lib.sdattn_qk_stats_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]

@@ -126,8 +126,10 @@ struct FlashCfg {
   static constexpr int V_TX = (DSLABS - 1) * KV_SLAB + TAIL * 2 * BN;   // bytes the V loads deliver
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int QBUF = 2;                  // Q tiles double-buffered across work units
+  static constexpr int OCW = D <= 80 ? D : 80;     // O columns per coalesced store pass
+  static constexpr int STG_BYTES = 4 * NQ * RowStage<OCW>::BYTES;   // one slice per softmax warp
   // 227 KB per CTA, less alignment slack, barriers and the tensor-memory word
-  static constexpr int STAGES_FIT = (232448 - 1024 - 16 - 8 * 32 - QBUF * NQ * Q_TILE) / STAGE;
+  static constexpr int STAGES_FIT = (232448 - 1024 - 16 - 8 * 32 - QBUF * NQ * Q_TILE - STG_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   // tensor memory per query tile: S (BN fp32), P (BN/2 columns of 16-bit pairs), O (PVN fp32)
   static constexpr uint32_t TM_S = 0;
@@ -137,7 +139,8 @@ struct FlashCfg {
   static constexpr uint32_t TMEM_COLS = NQ * QCOLS <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QBUF * NQ * Q_TILE;
-  static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
+  static constexpr int OFF_STG = OFF_KV + STAGES * STAGE;
+  static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
   static constexpr int NBAR = 2 * QBUF + 3 * STAGES + 5 * NQ + 2;
   static constexpr int MISC = 4 + 4 * NQ;   // words after the barriers
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + MISC * 4 + 1024;
@@ -150,6 +153,7 @@ struct FlashCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
   static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
+  static_assert(D % OCW == 0, "whole store passes");
 };
 
 // A unit whose key range is cut between two CTAs (split schedule) is
@@ -217,11 +221,12 @@ __device__ __forceinline__ uint32_t tile_count(uint32_t* ticket, uint32_t v, int
 // flags: two words, used once each.  Out of line: it runs at most twice per
 // CTA, and inlined it would weigh on the register allocation of the softmax
 // loop (the softmax warps hold more registers than any callee may use).
-template <int D, bool BF16, int ROWF>
+template <int D, int OCW, bool BF16, int ROWF>
 __device__ __noinline__ void flash_cut_epilogue(float* part, uint32_t* tickets, float* LS, int N, float scale,
                                                 float c, uint32_t o_tmem, int side, int64_t slot, int q, int r,
                                                 int bh, int row, float m_used, float l, float rawmax,
-                                                volatile uint32_t* flags, uint8_t* orow) {
+                                                volatile uint32_t* flags, uint8_t* slice, uint8_t* owarp,
+                                                int ovalid) {
   float4* mine = partial_rows<ROWF>(part, slot, side) + r;
   const float4* theirs = partial_rows<ROWF>(part, slot, side ^ 1) + r;
   constexpr int G = D / 8 < 5 ? D / 8 : 5;   // chunks of 8 columns per tensor-memory wait
@@ -263,6 +268,8 @@ __device__ __noinline__ void flash_cut_epilogue(float* part, uint32_t* tickets, 
   const float a_mine = side ? a_t : a_h, a_theirs = side ? a_h : a_t;
   const float lsum = fmaf(l_h, a_h, l_t * a_t);
   const float inv = 1.f / lsum;
+  const int lane = r & 31;
+  static_assert((OCW / 8) % G == 0, "column groups per store pass");
 #pragma unroll
   for (int g0 = 0; g0 < D / 8; g0 += G) {
     uint32_t o[8 * G];
@@ -288,8 +295,10 @@ __device__ __noinline__ void flash_cut_epilogue(float* part, uint32_t* tickets, 
       w.y = pack2<BF16>(f[2], f[3]);
       w.z = pack2<BF16>(f[4], f[5]);
       w.w = pack2<BF16>(f[6], f[7]);
-      if (row < N) *reinterpret_cast<uint4*>(orow + (g0 + i) * 16) = w;
+      stage_put<OCW>(slice, lane, (g0 + i) % (OCW / 8), w);
     }
+    if ((g0 + G) % (OCW / 8) == 0)   // a store pass is complete
+      stage_flush<OCW>(slice, lane, owarp + ((g0 + G) / (OCW / 8) - 1) * OCW * 2, D * 2, ovalid);
   }
   if (LS != nullptr && row < N) {
     const float raw = fmaxf(rawmax, t2.z);
@@ -606,25 +615,47 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
       if (!live) break;
       tc_fence_after();
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row) * D * 2;
+      // this warp's 32 rows of O: consecutive rows, stored through its shared-memory slice
+      const int row_w = row - lane;
+      uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * 2;
+      const int ovalid = p.N - row_w;
+      uint8_t* slice = smem + C::OFF_STG + (warp - 4) * RowStage<C::OCW>::BYTES;
       if (!(p.split && sg.cut(p))) {
-        // O's D columns and the row sum l (column D), one tensor-memory wait
-        uint32_t o[D + 8];
+        // O in store passes of OCW columns; the first pass also brings the row
+        // sum l (column D) when it fits beside them, all behind one wait
+        constexpr int NPASS = D / C::OCW;
+        constexpr int XL = NPASS == 1 ? 8 : 0;   // column D loaded with the only pass
+        float l = 0.f, inv = 0.f;
+        if constexpr (NPASS > 1) {
+          uint32_t t8[8];
+          tmem_ld_x8(o_tmem + D, t8);
+          tmem_wait_ld();
+          reg_fence<8>(t8);
+          l = __uint_as_float(t8[0]);
+          inv = 1.f / l;
+        }
 #pragma unroll
-        for (int c8 = 0; c8 <= D / 8; ++c8) tmem_ld_x8(o_tmem + c8 * 8, o + c8 * 8);
-        tmem_wait_ld();
-        reg_fence<D + 8>(o);
-        const float l = __uint_as_float(o[D]);
-        const float inv = 1.f / l;
+        for (int ps = 0; ps < NPASS; ++ps) {
+          uint32_t o[C::OCW + XL];
 #pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          const uint32_t* oc = o + c8 * 8;
-          uint4 w;
-          w.x = pack2<BF16>(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
-          w.y = pack2<BF16>(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
-          w.z = pack2<BF16>(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
-          w.w = pack2<BF16>(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
-          if (row < p.N) *reinterpret_cast<uint4*>(orow + c8 * 16) = w;
+          for (int c8 = 0; c8 < (C::OCW + XL) / 8; ++c8) tmem_ld_x8(o_tmem + ps * C::OCW + c8 * 8, o + c8 * 8);
+          tmem_wait_ld();
+          reg_fence<C::OCW + XL>(o);
+          if constexpr (NPASS == 1) {
+            l = __uint_as_float(o[D]);
+            inv = 1.f / l;
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < C::OCW / 8; ++c8) {
+            const uint32_t* oc = o + c8 * 8;
+            uint4 w;
+            w.x = pack2<BF16>(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+            w.y = pack2<BF16>(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+            w.z = pack2<BF16>(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+            w.w = pack2<BF16>(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
+            stage_put<C::OCW>(slice, lane, c8, w);
+          }
+          stage_flush<C::OCW>(slice, lane, owarp + ps * C::OCW * 2, D * 2, ovalid);
         }
         if (p.LS != nullptr && row < p.N) {
           const float L = rawmax * p.scale;
@@ -641,9 +672,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           l = __uint_as_float(o[0]);
         }
         const int side = sg.j0 > 0 ? 1 : 0;   // 0: head half, 1: tail half
-        flash_cut_epilogue<D, BF16, C::ROWF>(p.part, p.tickets, p.LS, p.N, p.scale, c, o_tmem, side,
-                                            static_cast<int64_t>(blockIdx.x - side) * NQ + q, q, r, bh, row, m_used,
-                                            l, rawmax, misc + 4 + 4 * q + 2 * kcut, orow);
+        flash_cut_epilogue<D, C::OCW, BF16, C::ROWF>(p.part, p.tickets, p.LS, p.N, p.scale, c, o_tmem, side,
+                                                    static_cast<int64_t>(blockIdx.x - side) * NQ + q, q, r, bh, row,
+                                                    m_used, l, rawmax, misc + 4 + 4 * q + 2 * kcut, slice, owarp,
+                                                    ovalid);
         ++kcut;
       }
       tc_fence_before();

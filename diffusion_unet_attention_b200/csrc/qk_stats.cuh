@@ -20,11 +20,22 @@
 // merged pair to the workspace and bumps an arrival counter; the unit that
 // arrives last merges all splits into LS, then zeroes the partials it read and
 // the counter (no spinning), so a completed call leaves the workspace zero.
+//
+// Store modes (template parameter AMODE):
+//   kAF32Stats  A in fp32 and the row statistics (the partially fused form);
+//   kAF32Only   A in fp32 only: the first pass of the three-pass form, whose
+//               statistics come from a separate kernel that reads A back
+//               (row_stats.cuh);
+//   kAF16Stats  A rounded to fp16 (half the bytes of A written and read), the
+//               statistics taken from the rounded values, so that the second
+//               kernel's exp(A_ij - L_i) sum to exactly S_i's terms.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace sdattn {
+
+enum QKMode : int { kAF32Stats = 0, kAF32Only = 1, kAF16Stats = 2 };
 
 struct QKParams {
   int N, M, BH;
@@ -82,7 +93,7 @@ __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2)
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, int AMODE>
 __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
     qk_stats_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const QKParams p) {
@@ -244,60 +255,83 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
         float a[128];
 #pragma unroll
         for (int k = 0; k < 128; ++k) a[k] = __uint_as_float(v[k]) * p.scale;
+        if constexpr (AMODE == kAF16Stats) {
+          // A is stored in fp16: the statistics are taken from the stored values
+#pragma unroll
+          for (int k = 0; k < 128; k += 2) {
+            const float2 r = __half22float2(__floats2half2_rn(a[k], a[k + 1]));
+            a[k] = r.x;
+            a[k + 1] = r.y;
+          }
+        }
         const int col0 = cb * 128;
         const int valid = min(128, p.M - col0);
-        // block partial (m_b, s_b) over the valid columns of this 128-column block
-        // eight independent chains for the max and for the sum, then a tree
-        float mx8[8], sm8[8];
-        if (valid == 128) {
+        if constexpr (AMODE != kAF32Only) {
+          // block partial (m_b, s_b) over the valid columns of this 128-column block
+          // eight independent chains for the max and for the sum, then a tree
+          float mx8[8], sm8[8];
+          if (valid == 128) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = fmax3(a[i], a[8 + i], a[16 + i]);
+            for (int i = 0; i < 8; ++i) mx8[i] = fmax3(a[i], a[8 + i], a[16 + i]);
 #pragma unroll
-          for (int k = 24; k < 128; k += 16)
+            for (int k = 24; k < 128; k += 16)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], a[k + i], (k + 8 + i < 128) ? a[k + 8 + i] : a[k + i]);
-        } else {
+              for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], a[k + i], (k + 8 + i < 128) ? a[k + 8 + i] : a[k + i]);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < 128; ++k) mx8[k & 7] = (k < valid) ? fmaxf(mx8[k & 7], a[k]) : mx8[k & 7];
+            for (int k = 0; k < 128; ++k) mx8[k & 7] = (k < valid) ? fmaxf(mx8[k & 7], a[k]) : mx8[k & 7];
+          }
+          const float mb =
+              fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], fmax3(mx8[5], mx8[6], mx8[7])));
+          const float nmb = -mb * L2E;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
+          if (valid == 128) {
+#pragma unroll
+            for (int k = 0; k < 128; ++k) sm8[k & 7] += ex2_approx(fmaf(a[k], L2E, nmb));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 128; ++k) sm8[k & 7] += (k < valid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
+          }
+          const float sb = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+          ms_merge(m_run, s_run, mb, sb);
         }
-        const float mb = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], fmax3(mx8[5], mx8[6], mx8[7])));
-        const float nmb = -mb * L2E;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
-        if (valid == 128) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k) sm8[k & 7] += ex2_approx(fmaf(a[k], L2E, nmb));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 128; ++k) sm8[k & 7] += (k < valid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
-        }
-        const float sb = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-        ms_merge(m_run, s_run, mb, sb);
 
-        // stream the block to A: 4 chunks of 32 columns x this warp's 32 rows
+        // stream the block to A: chunks of 128 bytes per row x this warp's 32
+        // rows (32 fp32 or 64 fp16 columns per chunk)
+        constexpr int CC = AMODE == kAF16Stats ? 64 : 32;   // columns per chunk
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (col0 + 32 * c >= p.M) break;
+        for (int c = 0; c < 128 / CC; ++c) {
+          if (col0 + CC * c >= p.M) break;
           uint8_t* buf = stg + (sc % C::NSTG) * C::STG;
           if (lane == 0) bulk_wait_read<C::NSTG - 1>();
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            float4 w = make_float4(a[32 * c + 4 * j + 0], a[32 * c + 4 * j + 1], a[32 * c + 4 * j + 2],
-                                   a[32 * c + 4 * j + 3]);
-            *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
+            uint4 w;
+            if constexpr (AMODE == kAF16Stats) {
+              const float* s8 = a + CC * c + 8 * j;
+              w = make_uint4(pack2<false>(s8[0], s8[1]), pack2<false>(s8[2], s8[3]), pack2<false>(s8[4], s8[5]),
+                             pack2<false>(s8[6], s8[7]));
+            } else {
+              const float* s4 = a + CC * c + 4 * j;
+              w = make_uint4(__float_as_uint(s4[0]), __float_as_uint(s4[1]), __float_as_uint(s4[2]),
+                             __float_as_uint(s4[3]));
+            }
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tmA, buf, col0 + 32 * c, rt * 128 + quarter * 32, bh);
+            tma_store_3d(&tmA, buf, col0 + CC * c, rt * 128 + quarter * 32, bh);
             bulk_commit();
           }
           ++sc;
         }
       }
+      if constexpr (AMODE == kAF32Only) continue;   // no statistics to finish
       // ---- the two groups' pairs merge; group 0 finishes the unit ----
       if (C::EPI == 2) {
         float2* slot = sMrg + (ui & 1) * 128;

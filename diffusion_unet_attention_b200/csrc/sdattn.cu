@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdlib>
@@ -15,6 +16,7 @@
 
 #include "flash.cuh"
 #include "qk_stats.cuh"
+#include "row_stats.cuh"
 #include "softmax_av.cuh"
 
 namespace {
@@ -25,6 +27,7 @@ using sdattn::FlashCfg;
 using sdattn::FlashParams;
 using sdattn::QKCfg;
 using sdattn::QKParams;
+using sdattn::RowStatsParams;
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplit = 16;
@@ -132,14 +135,19 @@ sdattn_status check_desc(const sdattn_desc* d) {
 
 int64_t a_ld(const sdattn_desc* d) { return (static_cast<int64_t>(d->M) + 3) / 4 * 4; }
 
+// Row stride of fp16-stored A, in elements: 16-byte rows.
+int64_t a16_ld(const sdattn_desc* d) { return (static_cast<int64_t>(d->M) + 7) / 8 * 8; }
+
 CUtensorMapDataType elem_type(const sdattn_desc* d) {
   return d->dtype == SDATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 }
 
 // Column splits of the statistics reduction: the smallest power of two that
-// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit,
-// and never below kMinBlocksPerSplit column blocks per split (each split
-// pays a partial write and an arrival, which a one-block split cannot hide).
+// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit.
+// A split keeps at least kMinBlocksPerSplit column blocks (each split pays a
+// partial write and an arrival, which a one-block split cannot hide on a busy
+// GPU), except while the doubled grid still fills at most half of the SMs:
+// there the shorter chain of blocks per CTA is worth more than the merge.
 struct QKPlan {
   int nrt, nb, nsplit, cbs, units;
 };
@@ -156,7 +164,9 @@ QKPlan plan_qk(const sdattn_desc* d, int nsm) {
   };
   int ns = 1;
   const int cap = pl.nb < kMaxSplit ? pl.nb : kMaxSplit;
-  while (ns * 2 <= cap && pl.nb / (ns * 2) >= kMinBlocksPerSplit && eff(base * ns) < 0.9) ns *= 2;
+  while (ns * 2 <= cap && (pl.nb / (ns * 2) >= kMinBlocksPerSplit || base * ns * 2 <= nsm / 2) &&
+         eff(base * ns) < 0.9)
+    ns *= 2;
   pl.cbs = (pl.nb + ns - 1) / ns;
   pl.nsplit = (pl.nb + pl.cbs - 1) / pl.cbs;
   pl.units = static_cast<int>(base * pl.nsplit);
@@ -193,35 +203,80 @@ size_t flash_ws_bytes(const sdattn_desc* d, int nsm) {
          static_cast<size_t>(nsm) * flash_nq_max(d->d) * 2 * 128 * rowf * sizeof(float);
 }
 
+// Stand-alone row statistics: one warp per (row, column split).  Rows are
+// split over several warps only while there are fewer rows than warps in a
+// persistent grid of two CTAs per SM, each split keeping at least 512 columns.
+struct RowPlan {
+  int64_t rows;
+  int nsplit, split_cols, grid;
+};
+
+RowPlan plan_rows(const sdattn_desc* d, int nsm) {
+  RowPlan pl;
+  pl.rows = static_cast<int64_t>(d->B) * d->H * d->N;
+  const int64_t warps = static_cast<int64_t>(nsm) * 2 * sdattn::kRowStatsWarps;
+  int ns = 1;
+  if (pl.rows < warps) {
+    const int64_t want = (warps + pl.rows - 1) / pl.rows;
+    const int64_t by_len = (d->M + 511) / 512;
+    ns = static_cast<int>(std::min<int64_t>(std::min<int64_t>(want, by_len), 64));
+    if (ns < 1) ns = 1;
+  }
+  pl.split_cols = static_cast<int>(((d->M + ns - 1) / ns + 31) / 32 * 32);
+  pl.nsplit = (d->M + pl.split_cols - 1) / pl.split_cols;
+  const int64_t items = pl.rows * pl.nsplit;
+  const int64_t ctas = (items + sdattn::kRowStatsWarps - 1) / sdattn::kRowStatsWarps;
+  pl.grid = static_cast<int>(std::min<int64_t>(ctas, static_cast<int64_t>(nsm) * 2));
+  return pl;
+}
+
+// [tickets: one uint32 per row, padded to 256 B][partials: float2 per (row, split)]
+size_t rows_ws_tickets_bytes(const RowPlan& pl) { return static_cast<size_t>((pl.rows * 4 + 255) / 256 * 256); }
+
+size_t rows_ws_bytes(const sdattn_desc* d, int nsm) {
+  const RowPlan pl = plan_rows(d, nsm);
+  if (pl.nsplit == 1) return 0;
+  return rows_ws_tickets_bytes(pl) + static_cast<size_t>(pl.rows) * pl.nsplit * sizeof(float2);
+}
+
 size_t ws_bytes(const sdattn_desc* d) {
   const int dev = current_device();
   const size_t qk = qk_ws_bytes(d);
-  const size_t fl = flash_ws_bytes(d, sm_count(dev < 0 ? 0 : dev));
-  return qk > fl ? qk : fl;
+  const int nsm = sm_count(dev < 0 ? 0 : dev);
+  const size_t fl = flash_ws_bytes(d, nsm);
+  const size_t rs = rows_ws_bytes(d, nsm);
+  return std::max(qk, std::max(fl, rs));
 }
 
 // --------------------------------------------------------------------------
 // Launchers
 // --------------------------------------------------------------------------
-template <int D, bool BF16>
-sdattn_status launch_qk(const sdattn_desc* d, const void* Q, const void* K, float* A, float* LS, void* ws,
+template <int D, bool BF16, int AMODE = sdattn::kAF32Stats>
+sdattn_status launch_qk(const sdattn_desc* d, const void* Q, const void* K, void* A, float* LS, void* ws,
                         cudaStream_t stream) {
   using C = QKCfg<D>;
   const int dev = current_device();
   if (dev < 0) return SDATTN_ERR_CUDA;
-  auto kern = sdattn::qk_stats_kernel<D, BF16>;
+  auto kern = sdattn::qk_stats_kernel<D, BF16, AMODE>;
   static std::atomic<uint64_t> smem_done{0};
   if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
 
   const int nsm = sm_count(dev);
   const QKPlan pl = plan_qk(d, nsm);
   const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
-  const uint64_t N = d->N, M = d->M, lda = a_ld(d);
+  const uint64_t N = d->N, M = d->M;
   CUtensorMap mq, mk, ma;
   if (!make_map_3d(&mq, Q, elem_type(d), D, N, bh, D * 2, N * D * 2, 64, 128)) return SDATTN_ERR_CUDA;
   if (!make_map_3d(&mk, K, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, 128)) return SDATTN_ERR_CUDA;
-  if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, N, bh, lda * 4, N * lda * 4, 32, 32))
-    return SDATTN_ERR_CUDA;
+  if constexpr (AMODE == sdattn::kAF16Stats) {
+    const uint64_t lda = a16_ld(d);
+    if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, M, N, bh, lda * 2, N * lda * 2, 64, 32))
+      return SDATTN_ERR_CUDA;
+  } else {
+    const uint64_t lda = a_ld(d);
+    if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, N, bh, lda * 4, N * lda * 4, 32, 32))
+      return SDATTN_ERR_CUDA;
+  }
 
   QKParams p;
   p.N = d->N;
@@ -240,22 +295,29 @@ sdattn_status launch_qk(const sdattn_desc* d, const void* Q, const void* K, floa
   return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, ma, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
-template <int D, bool BF16>
-sdattn_status launch_av(const sdattn_desc* d, const float* A, const float* LS, const void* V, void* O,
+template <int D, bool BF16, bool AF16 = false>
+sdattn_status launch_av(const sdattn_desc* d, const void* A, const float* LS, const void* V, void* O,
                         cudaStream_t stream) {
-  using C = AVCfg<D>;
+  using C = AVCfg<D, AF16>;
   const int dev = current_device();
   if (dev < 0) return SDATTN_ERR_CUDA;
-  auto kern = sdattn::softmax_av_kernel<D, BF16>;
+  auto kern = sdattn::softmax_av_kernel<D, BF16, AF16>;
   static std::atomic<uint64_t> smem_done{0};
   if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
 
   const int nsm = sm_count(dev);
   const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
-  const uint64_t N = d->N, M = d->M, lda = a_ld(d);
+  const uint64_t N = d->N, M = d->M;
   CUtensorMap ma, mv;
-  if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, N, bh, lda * 4, N * lda * 4, 32, 128))
-    return SDATTN_ERR_CUDA;
+  if constexpr (AF16) {
+    const uint64_t lda = a16_ld(d);
+    if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, M, N, bh, lda * 2, N * lda * 2, 64, 128))
+      return SDATTN_ERR_CUDA;
+  } else {
+    const uint64_t lda = a_ld(d);
+    if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, N, bh, lda * 4, N * lda * 4, 32, 128))
+      return SDATTN_ERR_CUDA;
+  }
   if (!make_map_3d(&mv, V, elem_type(d), D, M, bh, D * 2, M * D * 2, 64, C::BK)) return SDATTN_ERR_CUDA;
 
   AVParams p;
@@ -321,6 +383,64 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, mv, mvt, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
+sdattn_status launch_row_stats(const sdattn_desc* d, const float* A, float* LS, void* ws, size_t ws_size,
+                               cudaStream_t stream) {
+  const int dev = current_device();
+  const RowPlan pl = plan_rows(d, sm_count(dev < 0 ? 0 : dev));
+  RowStatsParams p;
+  p.A = A;
+  p.lda = a_ld(d);
+  p.rows = pl.rows;
+  p.M = d->M;
+  p.nsplit = pl.nsplit;
+  p.split_cols = pl.split_cols;
+  p.LS = LS;
+  p.tickets = nullptr;
+  p.part = nullptr;
+  if (pl.nsplit > 1) {
+    if (!ws || ws_size < rows_ws_tickets_bytes(pl) + static_cast<size_t>(pl.rows) * pl.nsplit * sizeof(float2))
+      return SDATTN_ERR_WORKSPACE;
+    p.tickets = static_cast<uint32_t*>(ws);
+    p.part = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + rows_ws_tickets_bytes(pl));
+  }
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  return launch(sdattn::row_stats_kernel<float>, pl.grid, sdattn::kRowStatsWarps * 32, 0, stream, p)
+             ? SDATTN_OK
+             : SDATTN_ERR_CUDA;
+}
+
+template <int AMODE>
+sdattn_status dispatch_qk(const sdattn_desc* d, const void* Q, const void* K, void* A, float* LS, void* ws,
+                          cudaStream_t s) {
+  const bool bf = d->dtype == SDATTN_BF16;
+  switch (d->d) {
+    case 40: return bf ? launch_qk<40, true, AMODE>(d, Q, K, A, LS, ws, s) : launch_qk<40, false, AMODE>(d, Q, K, A, LS, ws, s);
+    case 80: return bf ? launch_qk<80, true, AMODE>(d, Q, K, A, LS, ws, s) : launch_qk<80, false, AMODE>(d, Q, K, A, LS, ws, s);
+    case 160:
+      return bf ? launch_qk<160, true, AMODE>(d, Q, K, A, LS, ws, s) : launch_qk<160, false, AMODE>(d, Q, K, A, LS, ws, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
+}
+
+template <bool AF16>
+sdattn_status dispatch_av(const sdattn_desc* d, const void* A, const float* LS, const void* V, void* O,
+                          cudaStream_t s) {
+  const bool bf = d->dtype == SDATTN_BF16;
+  switch (d->d) {
+    case 40: return bf ? launch_av<40, true, AF16>(d, A, LS, V, O, s) : launch_av<40, false, AF16>(d, A, LS, V, O, s);
+    case 80: return bf ? launch_av<80, true, AF16>(d, A, LS, V, O, s) : launch_av<80, false, AF16>(d, A, LS, V, O, s);
+    case 160: return bf ? launch_av<160, true, AF16>(d, A, LS, V, O, s) : launch_av<160, false, AF16>(d, A, LS, V, O, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
+}
+
+// Work split of a qk_stats call with statistics: the scratch that its column
+// split needs (none for a single split).
+size_t qk_split_need(const sdattn_desc* d, const QKPlan& pl) {
+  const int64_t tiles = static_cast<int64_t>(d->B) * d->H * pl.nrt;
+  return pl.nsplit > 1 ? ws_tickets_bytes(d) + static_cast<size_t>(tiles) * 128 * pl.nsplit * sizeof(float2) : 0;
+}
+
 template <bool BF16>
 sdattn_status dispatch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
                              void* ws, cudaStream_t s) {
@@ -360,17 +480,51 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Process-unique id of the calling thread's current context (0 if none or
+// unknown).  A device reset ends the primary context; the next one has a new id.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // In host code `g_noalloc_scratch` only names the symbol; the device address
-// of the array is looked up once per device, with that device current.
+// of the array is looked up with the device current, once per device and
+// context: after a device reset the array lives in a new context, at an
+// address that is looked up anew.
 bool noalloc_scratch(int dev, void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   if (dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
     addr[dev] = p;
+    ctx_of[dev] = current_context_id();   // the lookup above made the primary context current
   }
   *out = addr[dev];
   return true;
@@ -401,33 +555,60 @@ sdattn_status sdattn_qk_stats(const sdattn_desc* desc, const void* Q, const void
   if (!aligned16(Q) || !aligned16(K) || !aligned16(A) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
   if (!ws || ws_size < qk_ws_bytes(desc)) return SDATTN_ERR_WORKSPACE;
   if (!aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool bf = desc->dtype == SDATTN_BF16;
-  switch (desc->d) {
-    case 40: return bf ? launch_qk<40, true>(desc, Q, K, A, LS, ws, s) : launch_qk<40, false>(desc, Q, K, A, LS, ws, s);
-    case 80: return bf ? launch_qk<80, true>(desc, Q, K, A, LS, ws, s) : launch_qk<80, false>(desc, Q, K, A, LS, ws, s);
-    case 160:
-      return bf ? launch_qk<160, true>(desc, Q, K, A, LS, ws, s) : launch_qk<160, false>(desc, Q, K, A, LS, ws, s);
-  }
-  return SDATTN_ERR_UNSUPPORTED;
+  return dispatch_qk<sdattn::kAF32Stats>(desc, Q, K, A, LS, ws, static_cast<cudaStream_t>(stream));
 }
 
 sdattn_status sdattn_softmax_av(const sdattn_desc* desc, const float* A, const float* LS, const void* V, void* O,
-                                void* ws, size_t ws_size, void* stream) {
+                                void* stream) {
   const sdattn_status st = check_desc(desc);
   if (st != SDATTN_OK) return st;
   if (!A || !LS || !V || !O) return SDATTN_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(LS) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
+  return dispatch_av<false>(desc, A, LS, V, O, static_cast<cudaStream_t>(stream));
+}
+
+sdattn_status sdattn_qk_scores(const sdattn_desc* desc, const void* Q, const void* K, float* A, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !A) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(A)) return SDATTN_ERR_ALIGNMENT;
+  return dispatch_qk<sdattn::kAF32Only>(desc, Q, K, A, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+sdattn_status sdattn_row_stats(const sdattn_desc* desc, const float* A, float* LS, void* ws, size_t ws_size,
+                               void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!A || !LS) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
   if (ws && !aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
   if (!ws && ws_size != 0) return SDATTN_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool bf = desc->dtype == SDATTN_BF16;
-  switch (desc->d) {
-    case 40: return bf ? launch_av<40, true>(desc, A, LS, V, O, s) : launch_av<40, false>(desc, A, LS, V, O, s);
-    case 80: return bf ? launch_av<80, true>(desc, A, LS, V, O, s) : launch_av<80, false>(desc, A, LS, V, O, s);
-    case 160: return bf ? launch_av<160, true>(desc, A, LS, V, O, s) : launch_av<160, false>(desc, A, LS, V, O, s);
-  }
-  return SDATTN_ERR_UNSUPPORTED;
+  return launch_row_stats(desc, A, LS, ws, ws_size, static_cast<cudaStream_t>(stream));
+}
+
+int64_t sdattn_a16_ld(const sdattn_desc* desc) {
+  if (check_desc(desc) != SDATTN_OK) return -1;
+  return a16_ld(desc);
+}
+
+sdattn_status sdattn_qk_stats_f16a(const sdattn_desc* desc, const void* Q, const void* K, void* A16, float* LS,
+                                   void* ws, size_t ws_size, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !A16 || !LS) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(A16) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
+  if (!ws || ws_size < qk_ws_bytes(desc)) return SDATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
+  return dispatch_qk<sdattn::kAF16Stats>(desc, Q, K, A16, LS, ws, static_cast<cudaStream_t>(stream));
+}
+
+sdattn_status sdattn_softmax_av_f16a(const sdattn_desc* desc, const void* A16, const float* LS, const void* V,
+                                     void* O, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!A16 || !LS || !V || !O) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(A16) || !aligned16(LS) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
+  return dispatch_av<true>(desc, A16, LS, V, O, static_cast<cudaStream_t>(stream));
 }
 
 sdattn_status sdattn_flash(const sdattn_desc* desc, const void* Q, const void* K, const void* V, void* O,
@@ -468,9 +649,7 @@ sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc* desc, const void* Q, co
   // Same work split as sdattn_qk_stats; a single split uses no scratch at all.
   const int dev = current_device();
   const QKPlan pl = plan_qk(desc, sm_count(dev < 0 ? 0 : dev));
-  const int64_t tiles = static_cast<int64_t>(desc->B) * desc->H * pl.nrt;
-  const size_t need =
-      pl.nsplit > 1 ? ws_tickets_bytes(desc) + static_cast<size_t>(tiles) * 128 * pl.nsplit * sizeof(float2) : 0;
+  const size_t need = qk_split_need(desc, pl);
   if (need > kNoAllocScratchBytes) return SDATTN_ERR_WORKSPACE;
   if (dev < 0) return SDATTN_ERR_CUDA;
   void* ws = nullptr;
@@ -478,14 +657,7 @@ sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc* desc, const void* Q, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The arrival counters must start at zero; the partials are overwritten.
   if (pl.nsplit > 1 && cudaMemsetAsync(ws, 0, ws_tickets_bytes(desc), s) != cudaSuccess) return SDATTN_ERR_CUDA;
-  const bool bf = desc->dtype == SDATTN_BF16;
-  switch (desc->d) {
-    case 40: return bf ? launch_qk<40, true>(desc, Q, K, A, LS, ws, s) : launch_qk<40, false>(desc, Q, K, A, LS, ws, s);
-    case 80: return bf ? launch_qk<80, true>(desc, Q, K, A, LS, ws, s) : launch_qk<80, false>(desc, Q, K, A, LS, ws, s);
-    case 160:
-      return bf ? launch_qk<160, true>(desc, Q, K, A, LS, ws, s) : launch_qk<160, false>(desc, Q, K, A, LS, ws, s);
-  }
-  return SDATTN_ERR_UNSUPPORTED;
+  return dispatch_qk<sdattn::kAF32Stats>(desc, Q, K, A, LS, ws, s);
 }
 
 const char* sdattn_status_string(sdattn_status status) {

@@ -428,6 +428,49 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Coalesced row stores.  An epilogue thread owns one output row (its tensor-
+// memory lane), so direct stores from a warp land 2*D bytes apart.  Instead a
+// warp puts its 32 rows (CW 16-bit columns of each, one pass) into its own
+// shared-memory slice, then stores the slice as consecutive 16-byte chunks:
+// the warp's rows are consecutive rows of O, so with CW = D one pass is one
+// contiguous block of 32 * 2D bytes.  The slice pitch is padded when a row
+// holds an even number of chunks, so that eight lanes storing one chunk of
+// eight different rows hit eight different bank groups.
+// ---------------------------------------------------------------------------
+template <int CW>
+struct RowStage {
+  static constexpr int NCH = CW / 8;                                   // 16-byte chunks per row
+  static constexpr int PITCH = (NCH % 2 == 0) ? NCH * 16 + 16 : NCH * 16;
+  static constexpr int BYTES = 32 * PITCH;                             // one warp's slice
+  static_assert(CW % 8 == 0, "whole 16-byte chunks");
+};
+
+// Lane `lane` puts chunk `ch` (columns 8ch .. 8ch+7 of this pass) of its row.
+template <int CW>
+__device__ __forceinline__ void stage_put(uint8_t* slice, int lane, int ch, uint4 w) {
+  *reinterpret_cast<uint4*>(slice + lane * RowStage<CW>::PITCH + ch * 16) = w;
+}
+
+// The warp stores its slice: rows r < valid_rows of the pass, row r at
+// grow0 + r * row_bytes (grow0: the warp's first row, first column of the
+// pass; 16-byte aligned).  Called by the whole warp after its stage_put calls.
+template <int CW>
+__device__ __forceinline__ void stage_flush(const uint8_t* slice, int lane, uint8_t* grow0, int row_bytes,
+                                            int valid_rows) {
+  using RS = RowStage<CW>;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < RS::NCH; ++i) {
+    const int c = i * 32 + lane;
+    const int r = c / RS::NCH, ch = c - r * RS::NCH;
+    if (r < valid_rows)
+      *reinterpret_cast<uint4*>(grow0 + static_cast<int64_t>(r) * row_bytes + ch * 16) =
+          *reinterpret_cast<const uint4*>(slice + r * RS::PITCH + ch * 16);
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31u) == 0u; }

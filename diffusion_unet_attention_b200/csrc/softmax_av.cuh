@@ -8,15 +8,16 @@
 // matrix is ever written.
 //
 // B200 design.  One persistent CTA per SM walks (b*H + h, 128-row tile) units.
-//   warp 0      TMA producer: a ring of (A block 128 x 64 fp32, V block 64 x d)
-//               stages, 128-byte swizzled;
+//   warp 0      TMA producer: a ring of (A block 128 x 64, fp32 or fp16, and V
+//               block 64 x d) stages, 128-byte swizzled;
 //   warps 2..5  one query row per thread: reads its 64 scores of the block from
 //               shared memory, computes p = exp(a - L_i) in registers, packs p
 //               to 16 bits and writes it to tensor memory (double-buffered);
 //   warp 1      tcgen05 MMA issuer: O += P V with P taken from tensor memory
 //               and V from shared memory, O accumulated in tensor memory.
-// The epilogue scales O by 1/S_i and stores it.  Since L_i is final, no
-// rescaling is ever needed.
+// The epilogue scales O by 1/S_i and stores it, each warp's 32 consecutive
+// rows through its own shared-memory slice as consecutive 16-byte chunks.
+// Since L_i is final, no rescaling is ever needed.
 #pragma once
 
 #include "sm100.cuh"
@@ -32,18 +33,20 @@ struct AVParams {
   void* O;
 };
 
-template <int D>
+template <int D, bool AF16 = false>
 struct AVCfg {
   static constexpr int DSLABS = (D + 63) / 64;
   static constexpr int PVN = DSLABS * 64;              // MMA N (head width padded to 64)
   static constexpr int BK = 64;                        // keys per block
-  static constexpr int A_BYTES = 128 * BK * 4;         // 32 KB: two 16 KB boxes of 32 fp32 columns
+  static constexpr int A_BYTES = 128 * BK * (AF16 ? 2 : 4);   // fp32: two 16 KB boxes of 32 columns; fp16: one of 64
   static constexpr int V_SLAB = BK * 128;              // 8 KB: 64 keys x 64 elements
   static constexpr int V_BYTES = DSLABS * V_SLAB;
   static constexpr int STAGES = D == 160 ? 3 : 4;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_V = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * V_BYTES;
+  static constexpr int OCW = D <= 80 ? D : 80;     // O columns per coalesced store pass
+  static constexpr int OFF_STG = OFF_V + STAGES * V_BYTES;   // one store slice per row warp
+  static constexpr int OFF_BAR = OFF_STG + 4 * RowStage<OCW>::BYTES;
   static constexpr int NBAR = 4 * STAGES + 4 + 1 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 256;
@@ -53,11 +56,11 @@ struct AVCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool AF16>
 __global__ void __launch_bounds__(192, 1)
     softmax_av_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
                       const AVParams p) {
-  using C = AVCfg<D>;
+  using C = AVCfg<D, AF16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + C::OFF_A;
@@ -123,7 +126,8 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(&v_empty[st], (n & 1) ^ 1, kSiteVEmpty, abort_flag)) { live = false; break; }
           mbar_arrive_expect_tx(&a_full[st], C::A_BYTES);
           tma_load_3d(sA + st * C::A_BYTES, &tmA, kb * C::BK, rt * 128, bh, &a_full[st]);
-          tma_load_3d(sA + st * C::A_BYTES + C::A_BYTES / 2, &tmA, kb * C::BK + 32, rt * 128, bh, &a_full[st]);
+          if constexpr (!AF16)
+            tma_load_3d(sA + st * C::A_BYTES + C::A_BYTES / 2, &tmA, kb * C::BK + 32, rt * 128, bh, &a_full[st]);
           mbar_arrive_expect_tx(&v_full[st], C::V_BYTES);
           for (int s = 0; s < C::DSLABS; ++s)
             tma_load_3d(sV + st * C::V_BYTES + s * C::V_SLAB, &tmV, 64 * s, kb * C::BK, bh, &v_full[st]);
@@ -188,28 +192,50 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t st = c % C::STAGES, n = c / C::STAGES;
         live = __all_sync(0xffffffffu, mbar_wait(&a_full[st], n & 1, kSiteAFull, abort_flag));
         if (!live) break;
-        // this row's 64 scores: two 32-column boxes, 128-byte swizzled rows
+        // this row's 64 scores, 128-byte swizzled rows: two 32-column fp32
+        // boxes, or one 64-column fp16 box
         uint32_t pk[32];
         const int valid = p.M - kb * C::BK;           // columns of this block inside [0, M)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint8_t* rowp = sA + st * C::A_BYTES + h * (C::A_BYTES / 2) + r * 128;
+        if constexpr (AF16) {
+          const uint8_t* rowp = sA + st * C::A_BYTES + r * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 a = *reinterpret_cast<const float4*>(rowp + ((j ^ (r & 7)) << 4));
-            const int k = h * 32 + 4 * j;
-            float e0 = ex2_approx(fmaf(a.x, L2E, nl));
-            float e1 = ex2_approx(fmaf(a.y, L2E, nl));
-            float e2 = ex2_approx(fmaf(a.z, L2E, nl));
-            float e3 = ex2_approx(fmaf(a.w, L2E, nl));
-            if (valid < C::BK) {
-              e0 = (k + 0 < valid) ? e0 : 0.f;
-              e1 = (k + 1 < valid) ? e1 : 0.f;
-              e2 = (k + 2 < valid) ? e2 : 0.f;
-              e3 = (k + 3 < valid) ? e3 : 0.f;
+            const uint4 h = *reinterpret_cast<const uint4*>(rowp + ((j ^ (r & 7)) << 4));
+            const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
+              const int k = 8 * j + 2 * i;
+              float e0 = ex2_approx(fmaf(a.x, L2E, nl));
+              float e1 = ex2_approx(fmaf(a.y, L2E, nl));
+              if (valid < C::BK) {
+                e0 = (k + 0 < valid) ? e0 : 0.f;
+                e1 = (k + 1 < valid) ? e1 : 0.f;
+              }
+              pk[k / 2] = pack2<BF16>(e0, e1);
             }
-            pk[k / 2 + 0] = pack2<BF16>(e0, e1);
-            pk[k / 2 + 1] = pack2<BF16>(e2, e3);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint8_t* rowp = sA + st * C::A_BYTES + h * (C::A_BYTES / 2) + r * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 a = *reinterpret_cast<const float4*>(rowp + ((j ^ (r & 7)) << 4));
+              const int k = h * 32 + 4 * j;
+              float e0 = ex2_approx(fmaf(a.x, L2E, nl));
+              float e1 = ex2_approx(fmaf(a.y, L2E, nl));
+              float e2 = ex2_approx(fmaf(a.z, L2E, nl));
+              float e3 = ex2_approx(fmaf(a.w, L2E, nl));
+              if (valid < C::BK) {
+                e0 = (k + 0 < valid) ? e0 : 0.f;
+                e1 = (k + 1 < valid) ? e1 : 0.f;
+                e2 = (k + 2 < valid) ? e2 : 0.f;
+                e3 = (k + 3 < valid) ? e3 : 0.f;
+              }
+              pk[k / 2 + 0] = pack2<BF16>(e0, e1);
+              pk[k / 2 + 1] = pack2<BF16>(e2, e3);
+            }
           }
         }
         __syncwarp();
@@ -231,19 +257,27 @@ __global__ void __launch_bounds__(192, 1)
       if (!live) break;
       tc_fence_after();
       const float inv = 1.f / Sr;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row) * D * 2;
+      const int row_w = row - lane;   // the warp's first row
+      uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * 2;
+      uint8_t* slice = smem + C::OFF_STG + (warp - 2) * RowStage<C::OCW>::BYTES;
 #pragma unroll
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        uint32_t o[8];
-        tmem_ld_x8(tmem + C::TM_O + c8 * 8 + lane_off, o);
+      for (int pass = 0; pass < D / C::OCW; ++pass) {
+        uint32_t o[C::OCW];
+#pragma unroll
+        for (int c8 = 0; c8 < C::OCW / 8; ++c8) tmem_ld_x8(tmem + C::TM_O + pass * C::OCW + c8 * 8 + lane_off, o + c8 * 8);
         tmem_wait_ld();
-        reg_fence<8>(o);
-        uint4 w;
-        w.x = pack2<BF16>(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
-        w.y = pack2<BF16>(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
-        w.z = pack2<BF16>(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
-        w.w = pack2<BF16>(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
-        if (row < p.N) *reinterpret_cast<uint4*>(orow + c8 * 16) = w;
+        reg_fence<C::OCW>(o);
+#pragma unroll
+        for (int c8 = 0; c8 < C::OCW / 8; ++c8) {
+          const uint32_t* oc = o + c8 * 8;
+          uint4 w;
+          w.x = pack2<BF16>(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+          w.y = pack2<BF16>(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+          w.z = pack2<BF16>(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+          w.w = pack2<BF16>(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
+          stage_put<C::OCW>(slice, lane, c8, w);
+        }
+        stage_flush<C::OCW>(slice, lane, owarp + pass * C::OCW * 2, D * 2, p.N - row_w);
       }
       tc_fence_before();
     }

@@ -18,6 +18,13 @@
  *      without writing A to memory.
  *      -> sdattn_flash
  *
+ * Variants of the partially fused form, measured against it:
+ *   - the page's reduction as a kernel of its own that reads A back
+ *     (three passes over A instead of two):
+ *      -> sdattn_qk_scores, sdattn_row_stats, sdattn_softmax_av
+ *   - A stored in fp16, halving the bytes of A written and read:
+ *      -> sdattn_qk_stats_f16a, sdattn_softmax_av_f16a
+ *
  * The page gives no formula for L and S.  This library reads them as
  *      L_i = max_j A_ij,     S_i = sum_j exp(A_ij - L_i)      (natural base)
  * with A = scale * Q K^T, so that softmax(A)_ij = exp(A_ij - L_i) / S_i.
@@ -31,6 +38,8 @@
  *        O  [B][H][N][d]      element type desc->dtype
  *        A  [B][H][N][lda]    float32, lda = sdattn_a_ld(desc) >= M; only the
  *                             first M entries of each row are read or written
+ *        A16 [B][H][N][lda16] float16 (the fp16-A variant), lda16 =
+ *                             sdattn_a16_ld(desc) >= M
  *        LS [B][H][N][2]      float32, (L_i, S_i) pairs
  *  - Every pointer must be 16-byte aligned.  Buffers must not overlap.
  *  - Calls only enqueue work on `stream` (a cudaStream_t, or NULL for the
@@ -87,12 +96,13 @@ typedef enum {
  * Returns -1 for an invalid descriptor. */
 int64_t sdattn_a_ld(const sdattn_desc *desc);
 
-/* Bytes of workspace that sdattn_qk_stats, sdattn_softmax_av and sdattn_flash
- * need for this shape on the current device (split-reduction partials plus
- * arrival counters): enough for each of the three calls.  The same workspace
- * serves all three calls and any shape whose need is at most its size.  It
- * must be zero-filled once before its first use; every completed call leaves
- * all of it zero again.  After SDATTN_ERR_TIMEOUT it must be zero-filled anew.
+/* Bytes of workspace that sdattn_qk_stats, sdattn_qk_stats_f16a,
+ * sdattn_row_stats and sdattn_flash need for this shape on the current device
+ * (split-reduction partials plus arrival counters): enough for each of these
+ * calls.  The same workspace serves all of them and any shape whose need is
+ * at most its size.  It must be zero-filled once before its first use; every
+ * completed call leaves all of it zero again.  After SDATTN_ERR_TIMEOUT it
+ * must be zero-filled anew.
  * Returns 0 for an invalid descriptor. */
 size_t sdattn_workspace_bytes(const sdattn_desc *desc);
 
@@ -112,13 +122,50 @@ sdattn_status sdattn_qk_stats(const sdattn_desc *desc, const void *Q, const void
 /* Partially fused softmax, second kernel: normalisation fused with the
  * multiplication by V.
  *   O[b][h][i][c] = (sum_j exp(A_ij - L_i) V[b][h][j][c]) / S_i
- * A, LS (as written by sdattn_qk_stats), V: inputs; O: output.
- * ws / ws_bytes: optional workspace (may be NULL / 0), reserved: this
- * version never splits a row's key range here and leaves a given workspace
- * untouched (a size without a pointer is still refused). */
+ * A, LS (as written by sdattn_qk_stats, or by sdattn_qk_scores followed by
+ * sdattn_row_stats), V: inputs; O: output.  Needs no workspace. */
 sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const float *LS,
-                                const void *V, void *O, void *ws, size_t ws_bytes,
-                                void *stream);
+                                const void *V, void *O, void *stream);
+
+/* Three-pass variant, first pass: the score matrix alone,
+ *   A[b][h][i][j] = scale * sum_k Q[b][h][i][k] K[b][h][j][k]   (fp32, j < M),
+ * bit for bit the A that sdattn_qk_stats writes.  Q, K: inputs; A: output.
+ * Needs no workspace. */
+sdattn_status sdattn_qk_scores(const sdattn_desc *desc, const void *Q, const void *K, float *A,
+                               void *stream);
+
+/* Three-pass variant, second pass: the page's stand-alone reduction of a
+ * materialised A to LS[b][h][i] = (L_i, S_i), reading A once (summary of the
+ * paper, partially fused softmax paragraph: blocks of A reduced to partial
+ * results, which are reduced to the final ones, one GPU command).  Each row,
+ * or each column split of a row when rows are few, is reduced by one warp
+ * with coalesced 16-byte loads and warp shuffles; the splits of a row are
+ * merged by the last one to finish.
+ * A: input (layout of sdattn_qk_stats' A); LS: output.  ws / ws_bytes: the
+ * workspace (zero-filled before first use, left zero by every completed
+ * call) of at least sdattn_workspace_bytes(desc) bytes; it may be NULL / 0
+ * when B*H*N is at least 32 times the SM count (no row is split then), and a
+ * split call without one returns SDATTN_ERR_WORKSPACE. */
+sdattn_status sdattn_row_stats(const sdattn_desc *desc, const float *A, float *LS, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* Row stride of fp16-stored A, in elements: M rounded up to a multiple of 8
+ * (16-byte rows).  Returns -1 for an invalid descriptor. */
+int64_t sdattn_a16_ld(const sdattn_desc *desc);
+
+/* fp16-A variant, first kernel: as sdattn_qk_stats, but A is rounded to fp16
+ * (nearest even) when stored, A16 = fp16(scale * Q K^T), and L, S are the
+ * statistics of the stored values (L_i = max_j A16_ij, S_i = sum_j
+ * exp(A16_ij - L_i)), so that the second kernel's weights sum to S_i.
+ * Q, K: inputs; A16 [B][H][N][sdattn_a16_ld(desc)] and LS: outputs; ws as
+ * for sdattn_qk_stats. */
+sdattn_status sdattn_qk_stats_f16a(const sdattn_desc *desc, const void *Q, const void *K, void *A16,
+                                   float *LS, void *ws, size_t ws_bytes, void *stream);
+
+/* fp16-A variant, second kernel: as sdattn_softmax_av, reading fp16 A16
+ * (as written by sdattn_qk_stats_f16a).  Needs no workspace. */
+sdattn_status sdattn_softmax_av_f16a(const sdattn_desc *desc, const void *A16, const float *LS,
+                                     const void *V, void *O, void *stream);
 
 /* FlashAttention form: one kernel, tiled over keys with an online softmax,
  * A never stored.  Q, K, V: inputs; O: output.  LS_or_null: if not NULL,
@@ -147,7 +194,9 @@ sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K
  * calls no allocating routine.
  *  - The first call on a device looks up the array's device address (once
  *    per device, with that device current); make that first call before any
- *    stream capture on the device.
+ *    stream capture on the device.  After a device reset (a new primary
+ *    context) the next call looks the address up again, so that first call
+ *    after the reset, too, belongs before any capture.
  *  - Each call clears the part of the array that must start at zero.  All
  *    calls share the one array, which keeps the last call's contents, so calls
  *    that may overlap on the GPU (different streams, different threads) race

@@ -24,7 +24,7 @@ def _desc(B=2, H=8, N=4096, M=4096, d=40, dtype=0, scale=0.158113883):
 def test_header_declarations_are_exported(lib):
     from diffusion_unet_attention_b200 import _lib
     hdr = open(os.path.join(ROOT, "include", "sdattn.h")).read()
-    declared = set(re.findall(r"\b(sdattn_[a-z_]+)\s*\(", hdr))
+    declared = set(re.findall(r"\b(sdattn_[a-z0-9_]+)\s*\(", hdr))
     assert declared == set(_lib.EXPORTS)
     for name in declared:
         assert hasattr(lib, name), name
@@ -33,6 +33,8 @@ def test_header_declarations_are_exported(lib):
 def test_a_ld_and_workspace(lib):
     for M, ld in [(4096, 4096), (77, 80), (1, 4), (64, 64), (129, 132)]:
         assert lib.sdattn_a_ld(ctypes.byref(_desc(M=M))) == ld
+    for M, ld in [(4096, 4096), (77, 80), (1, 8), (64, 64), (129, 136)]:
+        assert lib.sdattn_a16_ld(ctypes.byref(_desc(M=M))) == ld
     assert lib.sdattn_a_ld(ctypes.byref(_desc(d=64))) == -1
     ws = lib.sdattn_workspace_bytes(ctypes.byref(_desc()))
     # tickets for 2*8*32 row tiles plus 16 splits of 128 float2 per tile
@@ -49,7 +51,12 @@ def test_bad_descriptor(lib, kw, status):
     p = ctypes.c_void_p(4096)
     assert lib.sdattn_flash(ctypes.byref(d), p, p, p, p, None, None, 0, None) == status
     assert lib.sdattn_qk_stats(ctypes.byref(d), p, p, p, p, p, 1 << 30, None) == status
-    assert lib.sdattn_softmax_av(ctypes.byref(d), p, p, p, p, None, 0, None) == status
+    assert lib.sdattn_softmax_av(ctypes.byref(d), p, p, p, p, None) == status
+    assert lib.sdattn_qk_scores(ctypes.byref(d), p, p, p, None) == status
+    assert lib.sdattn_row_stats(ctypes.byref(d), p, p, p, 1 << 30, None) == status
+    assert lib.sdattn_qk_stats_f16a(ctypes.byref(d), p, p, p, p, p, 1 << 30, None) == status
+    assert lib.sdattn_softmax_av_f16a(ctypes.byref(d), p, p, p, p, None) == status
+    assert lib.sdattn_a16_ld(ctypes.byref(d)) == -1
 
 
 def test_null_and_misaligned_pointers(lib):
@@ -60,9 +67,16 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.sdattn_flash(ctypes.byref(d), None, ok, ok, ok, None, None, 0, None) == 1
     assert lib.sdattn_flash(ctypes.byref(d), ok, ok, bad, ok, None, None, 0, None) == 3
     assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, bad, None, 0, None) == 3
-    assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, None, None, 0, None) == 1
-    assert lib.sdattn_softmax_av(ctypes.byref(d), bad, ok, ok, ok, None, 0, None) == 3
+    assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, None, None) == 1
+    assert lib.sdattn_softmax_av(ctypes.byref(d), bad, ok, ok, ok, None) == 3
     assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, bad, ok, 1 << 30, None) == 3
+    assert lib.sdattn_qk_scores(ctypes.byref(d), ok, None, ok, None) == 1
+    assert lib.sdattn_qk_scores(ctypes.byref(d), ok, ok, bad, None) == 3
+    assert lib.sdattn_row_stats(ctypes.byref(d), ok, None, ok, 1 << 30, None) == 1
+    assert lib.sdattn_row_stats(ctypes.byref(d), bad, ok, ok, 1 << 30, None) == 3
+    assert lib.sdattn_qk_stats_f16a(ctypes.byref(d), ok, ok, bad, ok, ok, 1 << 30, None) == 3
+    assert lib.sdattn_softmax_av_f16a(ctypes.byref(d), ok, ok, None, ok, None) == 1
+    assert lib.sdattn_softmax_av_f16a(ctypes.byref(d), ok, ok, ok, bad, None) == 3
 
 
 def test_workspace_checked(lib):
@@ -71,7 +85,13 @@ def test_workspace_checked(lib):
     need = lib.sdattn_workspace_bytes(ctypes.byref(d))
     assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, None, need, None) == 4
     assert lib.sdattn_qk_stats(ctypes.byref(d), ok, ok, ok, ok, ok, 4096, None) == 4
-    assert lib.sdattn_softmax_av(ctypes.byref(d), ok, ok, ok, ok, None, 16, None) == 4
+    assert lib.sdattn_qk_stats_f16a(ctypes.byref(d), ok, ok, ok, ok, ok, 4096, None) == 4
+    # row statistics: the workspace is needed only when rows are split (few
+    # rows); a size without a pointer is always refused
+    assert lib.sdattn_row_stats(ctypes.byref(d), ok, ok, None, 16, None) == 4
+    few = _desc(B=1, H=1, N=16, M=4096)
+    assert lib.sdattn_row_stats(ctypes.byref(few), ok, ok, None, 0, None) == 4
+    assert lib.sdattn_workspace_bytes(ctypes.byref(few)) >= 16 * 8 * 8
     # flash: the workspace is optional, but a size without a pointer, a short
     # one or a misaligned one is refused before anything is enqueued
     bad = ctypes.c_void_p((1 << 20) + 8)

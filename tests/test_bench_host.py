@@ -27,15 +27,26 @@ def test_job_throughput_counts_every_rank():
 
 
 def test_traffic_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
-    digest = bench.source_digest()
-    good = tmp_path / "good.md"
-    good.write_text(f"text\n\ntraffic_bytes_per_launch: 15799552 (source {digest})\n")
-    monkeypatch.setattr(bench, "PROFILE_MD", str(good))
-    assert bench.profiled_traffic() == 15799552.0
-    stale = tmp_path / "stale.md"
-    stale.write_text("traffic_bytes_per_launch: 15799552 (source 0123456789abcdef)\n")
-    monkeypatch.setattr(bench, "PROFILE_MD", str(stale))
-    assert bench.profiled_traffic() is None
-    monkeypatch.setattr(bench, "PROFILE_MD", str(tmp_path / "missing.md"))
-    assert bench.profiled_traffic() is None
+    import json
+    for kernel in ("flash", "qk_stats", "softmax_av"):
+        digest = bench.source_digest(kernel)
+        good = tmp_path / f"{kernel}.json"
+        good.write_text(json.dumps({"source_digest": digest, "dram_bytes_read": 15799552, "dram_bytes_write": 0}))
+        monkeypatch.setitem(bench.PROFILE_JSON, kernel, str(good))
+        assert bench.profiled_traffic(kernel) == 15799552.0
+        stale = tmp_path / f"{kernel}_stale.json"
+        stale.write_text(json.dumps({"source_digest": "0123456789abcdef", "dram_bytes_read": 1,
+                                     "dram_bytes_write": 0}))
+        monkeypatch.setitem(bench.PROFILE_JSON, kernel, str(stale))
+        assert bench.profiled_traffic(kernel) is None
+        monkeypatch.setitem(bench.PROFILE_JSON, kernel, str(tmp_path / "missing.json"))
+        assert bench.profiled_traffic(kernel) is None
+    # each kernel's digest covers its own sources
+    assert len({bench.source_digest(k) for k in ("flash", "qk_stats", "softmax_av")}) == 3
 
+
+def test_both_arms_print_the_same_config():
+    cfg = bench.job_config(1)
+    assert cfg["flops_per_step"] == bench.STEP_FLOPS and cfg["calls_per_step"] == 32
+    assert bench.SET_BYTES > 126e6          # each input set is larger than the L2
+    assert bench.job_config(1) == cfg

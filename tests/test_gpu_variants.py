@@ -1,0 +1,121 @@
+"""GPU parity of the partially fused form's variants against the fp64 oracle.
+
+* Three passes: `qk_scores` writes A alone (bit for bit the A of
+  `qk_stats`), the stand-alone reduction `row_stats` reads it back into LS,
+  `softmax_av` finishes.  L within 1e-4 absolute and S within 1e-4 relative of
+  the oracle (fp32 sums of exact fp16 products and fp32 exponentials), O at
+  the gate (max |O - O_ref| <= 2e-3, ||O - O_ref||_F / ||O_ref||_F <= 1e-3).
+* fp16-stored A: A16 is the fp16 rounding (nearest even) of the fp32 A, L is
+  the row max of A16 exactly and S the sum of exp(A16 - L) (checked against
+  the oracle run on A16's own values, which pins the statistics to the stored
+  matrix); O against the exact oracle at the gate.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import diffusion_unet_attention_b200 as sd  # noqa: E402
+
+DEV = torch.device("cuda:0")
+MAX_ABS, REL_FROB = 2e-3, 1e-3
+L_TOL, S_RTOL = 1e-4, 1e-4
+
+
+def f32(x):
+    return float(np.float32(x))
+
+
+def o_err(got, ref):
+    diff = np.asarray(got, np.float64) - ref
+    return float(np.abs(diff).max()), float(np.linalg.norm(diff) / np.linalg.norm(ref))
+
+
+def gate(got, ref, what):
+    ea, er = o_err(got, ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    assert ea <= MAX_ABS and er <= REL_FROB, f"{what}: max_abs {ea:.3e} rel_frob {er:.3e}"
+    return ea, er
+
+
+SHAPES = [(1, 1, 256, 256, 40), (2, 8, 4096, 77, 40), (2, 8, 1024, 1024, 80), (2, 8, 256, 256, 160),
+          (2, 8, 64, 64, 160), (1, 2, 129, 129, 40), (2, 1, 300, 77, 80), (1, 3, 257, 200, 160),
+          (1, 1, 1, 1, 40), (1, 1, 16, 4096, 40), (3, 1, 70, 65, 40), (1, 1, 2, 3, 160)]
+
+
+def _inputs(B, H, N, M, d, seed=90):
+    q, k, v = synth.make_qkv(synth.Shape("v", B, H, N, M, d), seed + N % 5, call_id=M % 7)
+    return q, k, v, f32(1 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("B,H,N,M,d", SHAPES)
+def test_three_pass(B, H, N, M, d):
+    q, k, v, scale = _inputs(B, H, N, M, d)
+    rows = np.arange(N) if N <= 1024 else np.arange(0, N, 7)
+    ref = oracle.attention(q[:, :, rows], k, v, scale)
+    tq, tk, tv = (torch.from_numpy(x).to(DEV) for x in (q, k, v))
+    desc = sd.make_desc(B, H, N, M, d, torch.float16, scale)
+    ws = torch.zeros(sd.workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    a = sd.qk_scores(tq, tk, scale)
+    a_ref, ls_fused = sd.qk_stats(tq, tk, scale, ws=ws)
+    ls = sd.row_stats(a, M, d, ws=ws)
+    ls2 = sd.row_stats(a, M, d, ws=ws)
+    o = sd.softmax_av(a, ls, tv, scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a[..., :M], a_ref[..., :M]), "qk_scores must write qk_stats' A"
+    assert torch.equal(ls, ls2), "row_stats must be deterministic"
+    assert int(torch.count_nonzero(ws)) == 0, "workspace left dirty"
+    ls_h = ls[:, :, rows].cpu().numpy().astype(np.float64)
+    assert np.abs(ls_h[..., 0] - ref["L"]).max() <= L_TOL
+    assert np.abs(ls_h[..., 1] / ref["S"] - 1).max() <= S_RTOL
+    # the stand-alone reduction and the fused epilogue agree on L exactly
+    assert torch.equal(ls[..., 0], ls_fused[..., 0])
+    gate(o[:, :, rows].float().cpu().numpy(), ref["O"], "three-pass O")
+
+
+@pytest.mark.parametrize("B,H,N,M,d", SHAPES)
+def test_f16_stored_a(B, H, N, M, d):
+    q, k, v, scale = _inputs(B, H, N, M, d)
+    rows = np.arange(N) if N <= 1024 else np.arange(0, N, 7)
+    ref = oracle.attention(q[:, :, rows], k, v, scale)
+    tq, tk, tv = (torch.from_numpy(x).to(DEV) for x in (q, k, v))
+    a32, _ = sd.qk_stats(tq, tk, scale)
+    a16, ls = sd.qk_stats_f16a(tq, tk, scale)
+    o = sd.softmax_av_f16a(a16, ls, tv, scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a16[..., :M], a32[..., :M].half()), "A16 must be fp16(A)"
+    a16_h = a16[:, :, rows, :M].float().cpu().numpy().astype(np.float64)
+    ls_h = ls[:, :, rows].cpu().numpy().astype(np.float64)
+    assert np.array_equal(ls_h[..., 0], a16_h.max(axis=-1)), "L must be the row max of the stored A16"
+    s16 = np.exp(a16_h - a16_h.max(axis=-1, keepdims=True)).sum(axis=-1)
+    assert np.abs(ls_h[..., 1] / s16 - 1).max() <= S_RTOL
+    ea, er = gate(o[:, :, rows].float().cpu().numpy(), ref["O"], "fp16-A O")
+    print(f"fp16 A {B, H, N, M, d}: max_abs {ea:.3e} rel_frob {er:.3e}")
+
+
+def test_variants_on_64x64_self_sampled():
+    """Full-size 64x64-latent self-attention, every tile sampled."""
+    shape = synth.WORKLOADS["self64"]
+    q, k, v = synth.make_qkv(shape, synth.STREAM["self64"])
+    scale = f32(1 / math.sqrt(40))
+    rows = np.unique(np.concatenate([np.arange(0, 4096, 61), np.arange(127, 4096, 128), [4095]]))
+    ref = oracle.attention(q[:, :, rows], k, v, scale)
+    tq, tk, tv = (torch.from_numpy(x).to(DEV) for x in (q, k, v))
+    idx = torch.from_numpy(rows).to(DEV)
+    for variant in ("three_pass", "f16a"):
+        o = sd.partially_fused(tq, tk, tv, scale, variant=variant)
+        torch.cuda.synchronize()
+        ea, er = gate(o[:, :, idx].float().cpu().numpy(), ref["O"], variant)
+        print(f"{variant} 64x64 self: max_abs {ea:.3e} rel_frob {er:.3e}")
+        del o
+    status, detail = sd.device_error()
+    assert status == "SDATTN_OK", (status, hex(detail))

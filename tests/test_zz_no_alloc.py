@@ -4,7 +4,11 @@ It serves callers that may not allocate device memory (no workspace of their
 own): its split-reduction scratch is a fixed array inside the library.  These
 checks call it through the C ABI and compare it with sdattn_qk_stats (given a
 caller-owned workspace) on the same inputs, twice in a row, since every call
-reuses the one array that the previous call left behind.
+reuses the one array that the previous call left behind.  Both entry points
+run the same kernel with the same work split, and the split merge has a fixed
+order, so A and LS must be bitwise identical.  The cases run from the most
+column splits to none, so a call always finds the array as a call with a
+different layout left it.
 
 This file is named to be collected last, so that a run stopping at the first
 failure has already run every other test; it also passes on its own.
@@ -26,7 +30,6 @@ if not torch.cuda.is_available():
 from diffusion_unet_attention_b200 import _lib  # noqa: E402
 
 DEV = torch.device("cuda:0")
-A_TOL, L_TOL, S_RTOL = 1e-4, 1e-4, 1e-4      # the parity tolerances of the other GPU tests
 
 
 def _run(lib, fn, desc, tq, tk, lda, ws=None):
@@ -45,11 +48,13 @@ def _run(lib, fn, desc, tq, tk, lda, ws=None):
     return a, ls
 
 
+# Column splits with 148 SMs in brackets (the plan depends on the SM count).
 @pytest.mark.parametrize("B,H,N,M,d", [
-    (1, 1, 256, 4096, 40),      # 16 column splits: the scratch carries partials and counters
-    (2, 8, 4096, 4096, 40),     # 64x64-latent self-attention (2 splits)
-    (2, 8, 1024, 1024, 80),     # 32x32-latent self-attention
-    (2, 8, 300, 77, 160),       # a single split: no scratch in use
+    (1, 4, 128, 8192, 40),      # [16 splits] four row tiles of partials and counters
+    (2, 8, 512, 4096, 40),      # [8 splits]
+    (2, 8, 4096, 4096, 40),     # [2 splits] 64x64-latent self-attention
+    (2, 8, 1024, 1024, 80),     # [2 splits] 32x32-latent self-attention
+    (2, 8, 300, 77, 160),       # [1 split] no scratch in use
 ])
 def test_matches_workspace_entry_point_twice(B, H, N, M, d):
     lib = _lib.load()
@@ -59,21 +64,30 @@ def test_matches_workspace_entry_point_twice(B, H, N, M, d):
     lda = lib.sdattn_a_ld(ctypes.byref(desc))
     ws = torch.zeros(max(lib.sdattn_workspace_bytes(ctypes.byref(desc)), 256), dtype=torch.uint8, device=DEV)
     a_ref, ls_ref = _run(lib, "qk_stats", desc, tq, tk, lda, ws)
+    assert torch.isfinite(a_ref[..., :M]).all() and torch.isfinite(ls_ref).all()
     for _ in range(2):
         a, ls = _run(lib, "noalloc", desc, tq, tk, lda)
-        assert torch.isfinite(a[..., :M]).all() and torch.isfinite(ls).all()
-        assert (a[..., :M] - a_ref[..., :M]).abs().max().item() <= A_TOL
-        assert (ls[..., 0] - ls_ref[..., 0]).abs().max().item() <= L_TOL
-        assert ((ls[..., 1] / ls_ref[..., 1]) - 1).abs().max().item() <= S_RTOL
+        assert torch.equal(a[..., :M], a_ref[..., :M])
+        assert torch.equal(ls, ls_ref)
     status = ctypes.c_uint32(0)
     assert lib.sdattn_device_error(ctypes.byref(status)) == 0
 
 
 def test_rejects_shapes_beyond_its_scratch():
-    # 149 row tiles of an 8192-key row split 16 ways need about 2.4 MB of partials
+    """149 row tiles of 8192-key rows: with 148 SMs the plan splits each row 16
+    ways, whose partials (about 2.4 MB) exceed the 2 MiB array.  The split plan
+    follows the SM count, so the case is only known to exceed it on 148 SMs.
+    The buffers are real and full-size, so a call that were accepted would
+    still stay inside them."""
+    if torch.cuda.get_device_properties(DEV).multi_processor_count != 148:
+        pytest.skip("the split plan of this shape is worked out for 148 SMs")
     lib = _lib.load()
-    desc = _lib.Desc(1, 149, 128, 8192, 40, _lib.SDATTN_F16, 0.15811388)
-    p = torch.empty(16, dtype=torch.float32, device=DEV)
-    st = lib.sdattn_qk_stats_noalloc(ctypes.byref(desc), p.data_ptr(), p.data_ptr(), p.data_ptr(), p.data_ptr(),
+    B, H, N, M, d = 1, 149, 128, 8192, 40
+    desc = _lib.Desc(B, H, N, M, d, _lib.SDATTN_F16, 0.15811388)
+    q = torch.zeros((B, H, N, d), dtype=torch.float16, device=DEV)
+    k = torch.zeros((B, H, M, d), dtype=torch.float16, device=DEV)
+    a = torch.empty((B, H, N, M), dtype=torch.float32, device=DEV)
+    ls = torch.empty((B, H, N, 2), dtype=torch.float32, device=DEV)
+    st = lib.sdattn_qk_stats_noalloc(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), a.data_ptr(), ls.data_ptr(),
                                      None)
     assert _lib.STATUS[st] == "SDATTN_ERR_WORKSPACE"
