@@ -261,6 +261,18 @@ class Scratch:
             sd.flash(q, k, v, scale, out=o, ws=self.ws)
             return 1
         a, ls = self.views(call)
+        if form == "three_pass":
+            sd.qk_scores(q, k, scale, out_a=a)
+            sd.row_stats(a, call.M, call.d, q.dtype, out_ls=ls, ws=self.ws)
+            sd.softmax_av(a, ls, v, scale, out=o)
+            return 3
+        if form == "f16a":
+            lda16 = (call.M + 7) // 8 * 8
+            a16 = self.a.view(self.torch.float16)[:call.B * call.H * call.N * lda16]
+            a16 = a16.view(call.B, call.H, call.N, lda16)
+            sd.qk_stats_f16a(q, k, scale, out_a=a16, out_ls=ls, ws=self.ws)
+            sd.softmax_av_f16a(a16, ls, v, scale, out=o)
+            return 2
         sd.qk_stats(q, k, scale, out_a=a, out_ls=ls, ws=self.ws)
         sd.softmax_av(a, ls, v, scale, out=o)
         return 2
@@ -353,7 +365,8 @@ def run_gpu(args, rank, world, local_rank):
     e2e = None
     if rank == 0 and not args.no_side:
         extra = side_measurements(torch, sd, stream, sets, scratch, issue, K=min(K, 50))
-        extra["per_call"] = per_call_table(torch, sd, stream, sets[0], scratch)
+        extra["per_call"] = per_call_table(torch, sd, stream, sets, scratch)
+        extra["unet_ops"] = unet_ops_table(torch, sd, stream)
     if not args.no_side:
         # every rank feeds its own replica from host memory; the job's step is its slowest rank's
         barrier()
@@ -440,7 +453,12 @@ def side_measurements(torch, sd, stream, sets, scratch, issue, K):
     peaks, _ = measured_peaks()
     f_ms = time_graph(lambda s: issue(s, dom, lambda c: "flash"), K, len(dom))
     p_ms = time_graph(lambda s: issue(s, dom, lambda c: "partial"), max(K // 4, 5), len(dom))
-    pf_bytes = 2 * c2.a_bytes() + 4 * c2.B * c2.H * c2.N * c2.d * 2 + c2.B * c2.H * c2.N * 8
+    t3_ms = time_graph(lambda s: issue(s, dom, lambda c: "three_pass"), max(K // 4, 5), len(dom))
+    h_ms = time_graph(lambda s: issue(s, dom, lambda c: "f16a"), max(K // 4, 5), len(dom))
+    io = 4 * c2.B * c2.H * c2.N * c2.d * 2 + c2.B * c2.H * c2.N * 8
+    pf_bytes = 2 * c2.a_bytes() + io
+    t3_bytes = 3 * c2.a_bytes() + io + c2.B * c2.H * c2.N * 8
+    h_bytes = c2.a_bytes() + io
     out["kernels_64x64_self"] = {
         "flash": {"us": round(f_ms * 1e3, 2), "tflops": round(c2.flops / (f_ms * 1e-3) / 1e12, 1),
                   "frac_measured_tensor_peak": round(c2.flops / (f_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
@@ -448,54 +466,73 @@ def side_measurements(torch, sd, stream, sets, scratch, issue, K):
         "partially_fused": {"us": round(p_ms * 1e3, 2), "gbs": round(pf_bytes / (p_ms * 1e-3) / 1e9, 1),
                             "algorithmic_bytes": pf_bytes,
                             "frac_measured_hbm": round(pf_bytes / (p_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "three_pass": {"us": round(t3_ms * 1e3, 2), "gbs": round(t3_bytes / (t3_ms * 1e-3) / 1e9, 1),
+                       "algorithmic_bytes": t3_bytes,
+                       "frac_measured_hbm": round(t3_bytes / (t3_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                       "what": "qk_scores + row_stats (A read back) + softmax_av"},
+        "f16a": {"us": round(h_ms * 1e3, 2), "gbs": round(h_bytes / (h_ms * 1e-3) / 1e9, 1),
+                 "algorithmic_bytes": h_bytes,
+                 "frac_measured_hbm": round(h_bytes / (h_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                 "what": "qk_stats_f16a + softmax_av_f16a (A stored in fp16)"},
     }
     return out
 
 
-def per_call_table(torch, sd, stream, stepset, scratch, reps=15):
-    """Every distinct call of the step set in both forms, each timed alone with
-    CUDA events after an L2 flush (a 256 MB write), median of `reps`.  Rows
-    carry the call's algorithmic FLOPs and bytes, its fraction of the measured
-    tensor (flash) or HBM (partially fused) peak, and its time over its floor:
-    the larger of the FLOP floor, the byte floor and the measured time of a
-    minimal kernel launch timed the same way."""
+def per_call_table(torch, sd, stream, sets, scratch, reps=20):
+    """Every distinct call of the step set in both forms, and each partially
+    fused kernel alone: a CUDA graph of `reps` back-to-back launches of the
+    call (the two input sets alternating, as within a step) is replayed and
+    timed with CUDA events; time per call = replay time / reps.  Rows carry the
+    call's algorithmic FLOPs and bytes, its fraction of the measured tensor
+    (flash) or HBM (partially fused) peak, and its time over its floor: the
+    larger of the FLOP floor, the byte floor and the time per launch of a
+    minimal kernel timed the same way."""
     peaks, _ = measured_peaks()
     tflops_peak, hbm = float(peaks["bf16_tflops"]), float(peaks["hbm_gbs"])
-    dev = stepset.device
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    dev = sets[0].device
     tiny = torch.empty(4, dtype=torch.float32, device=dev)
     seen = {}
     for i, c in enumerate(CALLS):
         seen.setdefault((c.N, c.M, c.d), []).append(i)
 
-    def median_ms(fns):
-        """Per function in `fns` (issued back to back), the median time in ms."""
-        ts = [[] for _ in fns]
+    def per_launch_ms(issue_one):
+        g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
-            for _ in range(reps + 2):
-                flush.zero_()
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
-                ev[0].record(stream)
-                for j, fn in enumerate(fns):
-                    fn()
-                    ev[j + 1].record(stream)
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    issue_one(r)
+            for _ in range(2):
+                g.replay()
+            ts = []
+            for _ in range(3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
                 stream.synchronize()
-                for j in range(len(fns)):
-                    ts[j].append(ev[j].elapsed_time(ev[j + 1]))
-        return [statistics.median(t[2:]) for t in ts]
+                ts.append(a.elapsed_time(b) / reps)
+        del g
+        return statistics.median(ts)
 
-    launch_ms = median_ms([lambda: tiny.zero_()])[0]
+    launch_ms = per_launch_ms(lambda r: tiny.zero_())
     rows = []
     for (N, M, d), idxs in seen.items():
-        call, q, k, v, o = stepset.inputs[idxs[0]]
+        i = idxs[0]
+        call = CALLS[i]
         scale = 1.0 / math.sqrt(d)
         a, ls = scratch.views(call)
-        f_ms, = median_ms([lambda: sd.flash(q, k, v, scale, out=o, ws=scratch.ws)])
-        qk_ms, av_ms = median_ms([lambda: sd.qk_stats(q, k, scale, out_a=a, out_ls=ls, ws=scratch.ws),
-                                  lambda: sd.softmax_av(a, ls, v, scale, out=o)])
+        inp = [sets[r % 2].inputs[i] for r in range(2)]
+
+        def run(form):
+            return lambda r: scratch.run(*inp[r % 2], form)
+
+        f_ms = per_launch_ms(run("flash"))
+        p_ms = per_launch_ms(run("partial"))
+        qk_ms = per_launch_ms(lambda r: sd.qk_stats(inp[r % 2][1], inp[r % 2][2], scale, out_a=a, out_ls=ls,
+                                                    ws=scratch.ws))
+        av_ms = per_launch_ms(lambda r: sd.softmax_av(a, ls, inp[r % 2][3], scale, out=inp[r % 2][4]))
         io = 2 * call.B * call.H * (2 * call.N + 2 * call.M) * d          # Q, K, V read, O written
         pf_bytes = io + 2 * call.a_bytes() + 2 * 8 * call.B * call.H * call.N   # + A written, read; LS
-        p_ms = qk_ms + av_ms
         fl_floor = max(call.flops / (tflops_peak * 1e9), io / (hbm * 1e6), launch_ms)
         pf_floor = max(call.flops / (tflops_peak * 1e9), pf_bytes / (hbm * 1e6), 2 * launch_ms)
         rows.append({
@@ -510,8 +547,68 @@ def per_call_table(torch, sd, stream, stepset, scratch, reps=15):
                         "frac_hbm": round(pf_bytes / (p_ms * 1e-3) / 1e9 / hbm, 4),
                         "x_floor": round(p_ms / pf_floor, 2)},
         })
-    return {"launch_floor_us": round(launch_ms * 1e3, 2), "note": "each call alone after an L2 flush; "
-            "x_floor = time / max(FLOP floor, byte floor, minimal launch)", "rows": rows}
+    return {"launch_floor_us": round(launch_ms * 1e3, 2),
+            "note": f"graph replays of {reps} back-to-back launches of each call (two input sets alternating); "
+                    "x_floor = time / max(FLOP floor, byte floor, minimal launch)", "rows": rows}
+
+
+# The UNet's other specialised kernels at SD 1.4 512x512 shapes (B = 2):
+# GroupNorm (32 groups) at the four resolutions, the gated GELU over
+# 2 x h x w tokens with F = 4 x channels.
+GN_SHAPES = [(2, 320, 64, 64), (2, 640, 32, 32), (2, 1280, 16, 16), (2, 1280, 8, 8)]
+GEGLU_SHAPES = [(2 * 64 * 64, 1280), (2 * 32 * 32, 2560), (2 * 16 * 16, 5120), (2 * 8 * 8, 5120)]
+
+
+def unet_ops_table(torch, sd, stream, reps=40):
+    """GroupNorm and the gated GELU: each shape timed as a CUDA graph of `reps`
+    launches cycling over enough input/output buffers that their total exceeds
+    the L2 twice over (no launch finds its data in L2); bytes = input read once
+    + output written once."""
+    peaks, _ = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rows = []
+
+    def timed(issue, nbuf):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    issue(r % nbuf)
+            g.replay()
+            ts = []
+            for _ in range(3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                stream.synchronize()
+                ts.append(a.elapsed_time(b) / reps)
+        del g
+        return statistics.median(ts)
+
+    for (B, C, H, W) in GN_SHAPES:
+        nbytes = 2 * 2 * B * C * H * W
+        nbuf = max(2, math.ceil(256e6 / nbytes))
+        xs = [torch.randn(B, C, H, W, device=dev, dtype=torch.float16) for _ in range(nbuf)]
+        ys = [torch.empty_like(x) for x in xs]
+        gam, bet = torch.ones(C, device=dev), torch.zeros(C, device=dev)
+        ms = timed(lambda i: sd.group_norm(xs[i], gam, bet, 32, 1e-6, out=ys[i]), nbuf)
+        rows.append({"op": "group_norm", "shape": [B, C, H, W], "groups": 32, "us": round(ms * 1e3, 2),
+                     "mb": round(nbytes / 1e6, 2), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
+        del xs, ys
+    for (T, F) in GEGLU_SHAPES:
+        nbytes = 2 * T * 2 * F + 2 * T * F
+        nbuf = max(2, math.ceil(256e6 / nbytes))
+        xs = [torch.randn(T, 2 * F, device=dev, dtype=torch.float16) for _ in range(nbuf)]
+        ys = [torch.empty(T, F, device=dev, dtype=torch.float16) for _ in range(nbuf)]
+        ms = timed(lambda i: sd.geglu(xs[i], out=ys[i]), nbuf)
+        rows.append({"op": "geglu", "shape": [T, 2 * F], "us": round(ms * 1e3, 2), "mb": round(nbytes / 1e6, 2),
+                     "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
+        del xs, ys
+    return {"note": f"graph of {reps} launches over buffers totalling > 256 MB; fp16", "rows": rows}
 
 
 def end_to_end(torch, sd, stream, stepset, scratch, steps):

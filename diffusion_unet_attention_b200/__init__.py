@@ -13,7 +13,8 @@ three optimisations, attention-efficiency paragraphs):
 
 Variants of the partially fused form: the page's reduction as a kernel of its
 own over a stored A (`qk_scores`, `row_stats`, then `softmax_av`), and A
-stored in fp16 (`qk_stats_f16a`, `softmax_av_f16a`).
+stored in fp16 (`qk_stats_f16a`, `softmax_av_f16a`).  Beside attention, the
+two specialised UNet kernels of the same section: `group_norm` and `geglu`.
 
 This module only marshals torch tensors (device memory and streams) into the
 C ABI of libsdattn.so; all arithmetic runs in the CUDA kernels.  There is no
@@ -28,8 +29,8 @@ import torch
 
 from . import _lib
 
-__all__ = ["qk_stats", "softmax_av", "flash", "partially_fused", "qk_scores", "row_stats", "qk_stats_f16a",
-           "softmax_av_f16a", "device_error", "a_ld", "a16_ld", "workspace_bytes", "SdattnError", "load_library"]
+__all__ = ["qk_stats", "softmax_av", "flash", "flash_f32o", "partially_fused", "qk_scores", "row_stats", "qk_stats_f16a",
+           "softmax_av_f16a", "group_norm", "geglu", "device_error", "a_ld", "a16_ld", "workspace_bytes", "SdattnError", "load_library"]
 
 SdattnError = _lib.SdattnError
 load_library = _lib.load
@@ -258,6 +259,26 @@ def flash(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None
     return (O, LS) if (return_ls or out_ls is not None) else O
 
 
+def flash_f32o(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+               out: torch.Tensor | None = None, return_ls: bool = False):
+    """FlashAttention form with an fp32 O and P carried as two 16-bit parts:
+    the form that holds bf16 inputs to the fp16 accuracy bar.  Returns O
+    [B,H,N,d] float32 (and LS if asked)."""
+    B, H, N, M, d = _check_qk(q, k)
+    if v.shape != k.shape or v.dtype != q.dtype or not v.is_cuda:
+        raise ValueError("v must match k in shape and q in dtype")
+    q, k, v = _contig(q), _contig(k), _contig(v)
+    desc = make_desc(B, H, N, M, d, q.dtype, _scale(scale, d))
+    O = out if out is not None else torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if O.shape != (B, H, N, d) or O.dtype != torch.float32 or not O.is_contiguous():
+        raise ValueError("out must be contiguous fp32 [B,H,N,d]")
+    LS = torch.empty((B, H, N, 2), dtype=torch.float32, device=q.device) if return_ls else None
+    st = _lib_handle().sdattn_flash_f32o(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), O.data_ptr(),
+                                         LS.data_ptr() if LS is not None else None, _stream(q.device))
+    _lib.check("sdattn_flash_f32o", st)
+    return (O, LS) if return_ls else O
+
+
 def partially_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
                     variant: str = "fused"):
     """The partially fused form; returns O.
@@ -276,6 +297,47 @@ def partially_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: fl
         A, LS = qk_stats_f16a(q, k, scale)
         return softmax_av_f16a(A, LS, v, scale)
     raise ValueError(f"unknown variant {variant!r}")
+
+
+def group_norm(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, groups: int, eps: float = 1e-6,
+               out: torch.Tensor | None = None):
+    """Group normalisation of x [B, C, H, W] (fp16 or bf16, NCHW) with
+    per-channel fp32 gamma, beta [C], in one launch."""
+    if x.dim() != 4 or not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor [B, C, H, W]")
+    if x.dtype not in _DTYPES:
+        raise TypeError(f"dtype {x.dtype} not supported (float16 or bfloat16)")
+    B, C, H, W = x.shape
+    gamma = _contig(gamma.to(device=x.device, dtype=torch.float32))
+    beta = _contig(beta.to(device=x.device, dtype=torch.float32))
+    if gamma.shape != (C,) or beta.shape != (C,):
+        raise ValueError("gamma and beta must be [C]")
+    x = _contig(x)
+    Y = out if out is not None else torch.empty_like(x)
+    if Y.shape != x.shape or Y.dtype != x.dtype or not Y.is_contiguous():
+        raise ValueError("out must match x")
+    desc = _lib.GNDesc(B, C, H, W, int(groups), _DTYPES[x.dtype], float(eps))
+    st = _lib_handle().sdattn_group_norm(ctypes.byref(desc), x.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
+                                         Y.data_ptr(), _stream(x.device))
+    _lib.check("sdattn_group_norm", st)
+    return Y
+
+
+def geglu(x: torch.Tensor, out: torch.Tensor | None = None):
+    """The UNet's gated GELU: x [..., 2F] -> x[..., :F] * GELU(x[..., F:]) in one launch."""
+    if not x.is_cuda or x.dtype not in _DTYPES:
+        raise ValueError("x must be a float16 or bfloat16 CUDA tensor")
+    F = x.shape[-1] // 2
+    if x.shape[-1] != 2 * F:
+        raise ValueError("the last dimension must be even")
+    x = _contig(x)
+    T = x.numel() // (2 * F)
+    Y = out if out is not None else torch.empty(x.shape[:-1] + (F,), dtype=x.dtype, device=x.device)
+    if Y.numel() != T * F or Y.dtype != x.dtype or not Y.is_contiguous():
+        raise ValueError("out must hold x.shape[:-1] + (F,) values of x's dtype")
+    st = _lib_handle().sdattn_geglu(T, F, _DTYPES[x.dtype], x.data_ptr(), Y.data_ptr(), _stream(x.device))
+    _lib.check("sdattn_geglu", st)
+    return Y
 
 
 def device_error():

@@ -27,15 +27,22 @@ STATUS = {
 
 # Every symbol include/sdattn.h declares.
 EXPORTS = ("sdattn_a_ld", "sdattn_workspace_bytes", "sdattn_qk_stats", "sdattn_softmax_av", "sdattn_flash",
+           "sdattn_flash_f32o",
            "sdattn_qk_scores", "sdattn_row_stats", "sdattn_a16_ld", "sdattn_qk_stats_f16a",
-           "sdattn_softmax_av_f16a", "sdattn_qk_stats_noalloc", "sdattn_device_error", "sdattn_status_string",
-           "sdattn_version")
+           "sdattn_softmax_av_f16a", "sdattn_group_norm", "sdattn_geglu", "sdattn_qk_stats_noalloc",
+           "sdattn_device_error", "sdattn_status_string", "sdattn_version")
 
 
 class Desc(ctypes.Structure):
     """sdattn_desc: shape of one attention call."""
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("M", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class GNDesc(ctypes.Structure):
+    """sdattn_gn_desc: shape of one group normalisation."""
+    _fields_ = [("B", ctypes.c_int32), ("C", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("G", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eps", ctypes.c_float)]
 
 
 class SdattnError(RuntimeError):
@@ -66,6 +73,8 @@ def load(path: str = LIB_PATH):
     lib.sdattn_qk_stats.restype = ctypes.c_int
     lib.sdattn_softmax_av.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.sdattn_softmax_av.restype = ctypes.c_int
+    lib.sdattn_flash_f32o.argtypes = [dp, vp, vp, vp, vp, vp, vp]
+    lib.sdattn_flash_f32o.restype = ctypes.c_int
     lib.sdattn_qk_scores.argtypes = [dp, vp, vp, vp, vp]
     lib.sdattn_qk_scores.restype = ctypes.c_int
     lib.sdattn_row_stats.argtypes = [dp, vp, vp, vp, sz, vp]
@@ -78,6 +87,10 @@ def load(path: str = LIB_PATH):
     lib.sdattn_softmax_av_f16a.restype = ctypes.c_int
     lib.sdattn_flash.argtypes = [dp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.sdattn_flash.restype = ctypes.c_int
+    lib.sdattn_group_norm.argtypes = [ctypes.POINTER(GNDesc), vp, vp, vp, vp, vp]
+    lib.sdattn_group_norm.restype = ctypes.c_int
+    lib.sdattn_geglu.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
+    lib.sdattn_geglu.restype = ctypes.c_int
     lib.sdattn_qk_stats_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.sdattn_qk_stats_noalloc.restype = ctypes.c_int
     lib.sdattn_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]

@@ -31,6 +31,13 @@
 // The row sum l comes from the tensor core: V's padding column D holds 1 in
 // every stage (written once; the V tile loads never cover it), so column D of
 // O accumulates sum_j p_j from the same 16-bit P that multiplies V.
+//
+// Precise variant (template flag PREC, one query tile per CTA): P is carried
+// as a 16-bit high part plus the 16-bit rounding of its residual, P V runs as
+// two MMAs into the same accumulator, and O is written in fp32.  Both parts
+// have the input's type, so with bf16 inputs (8-bit mantissas) the weights
+// keep about 16 bits and the result meets the fp16 accuracy bar; a bf16 O
+// alone would round each output by up to 2^-9 of its value.
 #pragma once
 
 #include "sm100.cuh"
@@ -113,7 +120,7 @@ struct FlashSegments {
   __device__ __forceinline__ bool cut(const FlashParams& p) const { return j0 > 0 || j1 < p.nkv; }
 };
 
-template <int D, int NQ, int BN>
+template <int D, int NQ, int BN, bool PREC = false>
 struct FlashCfg {
   static constexpr int DSLABS = (D + 63) / 64;
   static constexpr int KSTEPS = (D + 15) / 16;
@@ -126,16 +133,20 @@ struct FlashCfg {
   static constexpr int V_TX = (DSLABS - 1) * KV_SLAB + TAIL * 2 * BN;   // bytes the V loads deliver
   static constexpr int STAGE = K_BYTES + V_BYTES;
   static constexpr int QBUF = 2;                  // Q tiles double-buffered across work units
-  static constexpr int OCW = D <= 80 ? D : 80;     // O columns per coalesced store pass
+  // O store passes, in 16-bit columns (an fp32 O column counts as two)
+  static constexpr int OCW = PREC ? 80 : (D <= 80 ? D : 80);
+  static constexpr int OPASS = (PREC ? 2 * D : D) / OCW;
   static constexpr int STG_BYTES = 4 * NQ * RowStage<OCW>::BYTES;   // one slice per softmax warp
   // 227 KB per CTA, less alignment slack, barriers and the tensor-memory word
   static constexpr int STAGES_FIT = (232448 - 1024 - 16 - 8 * 32 - QBUF * NQ * Q_TILE - STG_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
-  // tensor memory per query tile: S (BN fp32), P (BN/2 columns of 16-bit pairs), O (PVN fp32)
+  // tensor memory per query tile: S (BN fp32), P (BN/2 columns of 16-bit
+  // pairs; with PREC a second such buffer holds P's residual), O (PVN fp32)
   static constexpr uint32_t TM_S = 0;
   static constexpr uint32_t TM_P = BN;
-  static constexpr uint32_t TM_O = BN + BN / 2;
-  static constexpr int QCOLS = BN + BN / 2 + PVN;
+  static constexpr uint32_t TM_PL = BN + BN / 2;
+  static constexpr uint32_t TM_O = BN + (PREC ? BN : BN / 2);
+  static constexpr int QCOLS = TM_O + PVN;
   static constexpr uint32_t TMEM_COLS = NQ * QCOLS <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QBUF * NQ * Q_TILE;
@@ -153,7 +164,8 @@ struct FlashCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
   static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
-  static_assert(D % OCW == 0, "whole store passes");
+  static_assert((PREC ? 2 * D : D) % OCW == 0, "whole store passes");
+  static_assert(!PREC || NQ == 1, "the precise variant keeps one query tile per CTA");
 };
 
 // A unit whose key range is cut between two CTAs (split schedule) is
@@ -181,9 +193,9 @@ __device__ __forceinline__ float4* partial_rows(float* part, int64_t slot, int h
 
 // p = 2^(s*c - m) for one row's key tile, packed to 16-bit pairs: NPOLY of
 // every 8 pairs on the FMA pipe (exp2_poly2), the rest on MUFU.
-template <int BN, bool BF16, int NPOLY>
+template <int BN, bool BF16, int NPOLY, bool PREC = false>
 __device__ __forceinline__ void flash_exp_block(const uint32_t (&v)[BN], uint64_t c2, uint64_t nm2,
-                                                uint32_t (&pk)[BN / 2]) {
+                                                uint32_t (&pk)[BN / 2], uint32_t* pl = nullptr) {
 #pragma unroll
   for (int k = 0; k < BN / 2; ++k) {
     const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), c2, nm2);
@@ -196,6 +208,20 @@ __device__ __forceinline__ void flash_exp_block(const uint32_t (&v)[BN], uint64_
       e1 = ex2_approx(x1);
     }
     pk[k] = pack2<BF16>(e0, e1);
+    if constexpr (PREC) {
+      // the residual of the 16-bit rounding, itself rounded to 16 bits
+      float h0, h1;
+      if constexpr (BF16) {
+        const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[k]));
+        h0 = h.x;
+        h1 = h.y;
+      } else {
+        const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
+        h0 = h.x;
+        h1 = h.y;
+      }
+      pl[k] = pack2<BF16>(e0 - h0, e1 - h1);
+    }
   }
 }
 
@@ -315,12 +341,12 @@ __device__ __noinline__ void flash_cut_epilogue(float* part, uint32_t* tickets, 
   if (r == 0) tickets[slot] = 0u;
 }
 
-template <int D, int NQ, int BN, bool BF16, int NPOLY>
-__global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
+template <int D, int NQ, int BN, bool BF16, int NPOLY, bool PREC = false>
+__global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
     flash_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmVt,
                  const FlashParams p) {
-  using C = FlashCfg<D, NQ, BN>;
+  using C = FlashCfg<D, NQ, BN, PREC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -457,6 +483,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV) + C::K_BYTES, C::KV_SLAB, 1024);
     const uint32_t s_tm = tmem + q * C::QCOLS + C::TM_S;
     const uint32_t p_tm = tmem + q * C::QCOLS + C::TM_P;
+    const uint32_t pl_tm = tmem + q * C::QCOLS + C::TM_PL;
     const uint32_t o_tm = tmem + q * C::QCOLS + C::TM_O;
     uint32_t t_base = 0, kv_base = 0, ui = 0;
     bool live = true;
@@ -490,6 +517,10 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
             mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+          if constexpr (PREC) {
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) mma_ts(o_tm, pl_tm + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv, 1u);
+          }
           mma_commit(&pv_done[q]);
           mma_commit(&kv_empty[st]);
         }
@@ -510,6 +541,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_tmem = tmem + q * C::QCOLS + C::TM_S + lane_off;
     const uint32_t p_tmem = tmem + q * C::QCOLS + C::TM_P + lane_off;
+    const uint32_t pl_tmem = tmem + q * C::QCOLS + C::TM_PL + lane_off;
     const uint32_t o_tmem = tmem + q * C::QCOLS + C::TM_O + lane_off;
     const float c = p.c;
     uint32_t t = 0;        // tiles seen by this query-tile slot (all units)
@@ -570,6 +602,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         float alpha = 1.f;
         bool rescale = false;
         uint32_t pk[BN / 2];
+        uint32_t pl[PREC ? BN / 2 : 1];
         if (NQ == 2 && q == 0 && t == 0) {
           __syncwarp();
           if (lane == 0) mbar_arrive(stagger);
@@ -579,7 +612,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
           m_used = mt;
           rescale = (j > sg.j0);
         }
-        flash_exp_block<BN, BF16, NPOLY>(v, c2, f2_pack(-m_used, -m_used), pk);
+        flash_exp_block<BN, BF16, NPOLY, PREC>(v, c2, f2_pack(-m_used, -m_used), pk, pl);
         if (j > sg.j0) {
           // P V of the previous tile must be done: P is reused and O may be rescaled
           live = __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (t - 1) & 1, kSitePvDone, abort_flag));
@@ -601,9 +634,14 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         }
         if constexpr (BN == 128) {
           tmem_st_x64(p_tmem, pk);
+          if constexpr (PREC) tmem_st_x64(pl_tmem, pl);
         } else {
 #pragma unroll
           for (int cc = 0; cc < BN / 32; ++cc) tmem_st_x16(p_tmem + cc * 16, pk + cc * 16);
+          if constexpr (PREC) {
+#pragma unroll
+            for (int cc = 0; cc < BN / 32; ++cc) tmem_st_x16(pl_tmem + cc * 16, pl + cc * 16);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -616,15 +654,17 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
       if (!live) break;
       tc_fence_after();
       // this warp's 32 rows of O: consecutive rows, stored through its shared-memory slice
+      constexpr int EB = PREC ? 4 : 2;   // bytes per O element
       const int row_w = row - lane;
-      uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * 2;
+      uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * EB;
       const int ovalid = p.N - row_w;
       uint8_t* slice = smem + C::OFF_STG + (warp - 4) * RowStage<C::OCW>::BYTES;
       if (!(p.split && sg.cut(p))) {
-        // O in store passes of OCW columns; the first pass also brings the row
+        // O in store passes of PC columns; the first pass also brings the row
         // sum l (column D) when it fits beside them, all behind one wait
-        constexpr int NPASS = D / C::OCW;
-        constexpr int XL = NPASS == 1 ? 8 : 0;   // column D loaded with the only pass
+        constexpr int NPASS = C::OPASS;
+        constexpr int PC = C::OCW * 2 / EB;        // O columns per pass
+        constexpr int XL = NPASS == 1 ? 8 : 0;     // column D loaded with the only pass
         float l = 0.f, inv = 0.f;
         if constexpr (NPASS > 1) {
           uint32_t t8[8];
@@ -636,47 +676,55 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN>::NTHREADS, 1)
         }
 #pragma unroll
         for (int ps = 0; ps < NPASS; ++ps) {
-          uint32_t o[C::OCW + XL];
+          uint32_t o[PC + XL];
 #pragma unroll
-          for (int c8 = 0; c8 < (C::OCW + XL) / 8; ++c8) tmem_ld_x8(o_tmem + ps * C::OCW + c8 * 8, o + c8 * 8);
+          for (int c8 = 0; c8 < (PC + XL) / 8; ++c8) tmem_ld_x8(o_tmem + ps * PC + c8 * 8, o + c8 * 8);
           tmem_wait_ld();
-          reg_fence<C::OCW + XL>(o);
+          reg_fence<PC + XL>(o);
           if constexpr (NPASS == 1) {
             l = __uint_as_float(o[D]);
             inv = 1.f / l;
           }
 #pragma unroll
-          for (int c8 = 0; c8 < C::OCW / 8; ++c8) {
-            const uint32_t* oc = o + c8 * 8;
+          for (int ch = 0; ch < C::OCW / 8; ++ch) {   // 16-byte chunks of the pass
             uint4 w;
-            w.x = pack2<BF16>(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
-            w.y = pack2<BF16>(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
-            w.z = pack2<BF16>(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
-            w.w = pack2<BF16>(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
-            stage_put<C::OCW>(slice, lane, c8, w);
+            if constexpr (PREC) {
+              const uint32_t* oc = o + ch * 4;
+              w = make_uint4(__float_as_uint(__uint_as_float(oc[0]) * inv), __float_as_uint(__uint_as_float(oc[1]) * inv),
+                             __float_as_uint(__uint_as_float(oc[2]) * inv), __float_as_uint(__uint_as_float(oc[3]) * inv));
+            } else {
+              const uint32_t* oc = o + ch * 8;
+              w.x = pack2<BF16>(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv);
+              w.y = pack2<BF16>(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv);
+              w.z = pack2<BF16>(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv);
+              w.w = pack2<BF16>(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv);
+            }
+            stage_put<C::OCW>(slice, lane, ch, w);
           }
-          stage_flush<C::OCW>(slice, lane, owarp + ps * C::OCW * 2, D * 2, ovalid);
+          stage_flush<C::OCW>(slice, lane, owarp + ps * C::OCW * 2, D * EB, ovalid);
         }
         if (p.LS != nullptr && row < p.N) {
           const float L = rawmax * p.scale;
           const float S = l * ex2_approx(m_used - rawmax * c);
           *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(L, S);
         }
-      } else if (kcut < 2) {
-        float l;
-        {
-          uint32_t o[8];
-          tmem_ld_x8(o_tmem + D, o);
-          tmem_wait_ld();
-          reg_fence<8>(o);
-          l = __uint_as_float(o[0]);
+      } else if constexpr (!PREC) {
+        if (kcut < 2) {
+          float l;
+          {
+            uint32_t o[8];
+            tmem_ld_x8(o_tmem + D, o);
+            tmem_wait_ld();
+            reg_fence<8>(o);
+            l = __uint_as_float(o[0]);
+          }
+          const int side = sg.j0 > 0 ? 1 : 0;   // 0: head half, 1: tail half
+          flash_cut_epilogue<D, C::OCW, BF16, C::ROWF>(p.part, p.tickets, p.LS, p.N, p.scale, c, o_tmem, side,
+                                                      static_cast<int64_t>(blockIdx.x - side) * NQ + q, q, r, bh, row,
+                                                      m_used, l, rawmax, misc + 4 + 4 * q + 2 * kcut, slice, owarp,
+                                                      ovalid);
+          ++kcut;
         }
-        const int side = sg.j0 > 0 ? 1 : 0;   // 0: head half, 1: tail half
-        flash_cut_epilogue<D, C::OCW, BF16, C::ROWF>(p.part, p.tickets, p.LS, p.N, p.scale, c, o_tmem, side,
-                                                    static_cast<int64_t>(blockIdx.x - side) * NQ + q, q, r, bh, row,
-                                                    m_used, l, rawmax, misc + 4 + 4 * q + 2 * kcut, slice, owarp,
-                                                    ovalid);
-        ++kcut;
       }
       tc_fence_before();
     }

@@ -18,6 +18,7 @@
 #include "qk_stats.cuh"
 #include "row_stats.cuh"
 #include "softmax_av.cuh"
+#include "unet_ops.cuh"
 
 namespace {
 
@@ -333,13 +334,13 @@ sdattn_status launch_av(const sdattn_desc* d, const void* A, const float* LS, co
   return launch(kern, grid, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
-template <int D, int NQ, int BN, bool BF16, int NPOLY = 3>
+template <int D, int NQ, int BN, bool BF16, int NPOLY = 3, bool PREC = false>
 sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, const void* V, void* O, float* LS,
                            void* ws, cudaStream_t stream) {
-  using C = FlashCfg<D, NQ, BN>;
+  using C = FlashCfg<D, NQ, BN, PREC>;
   const int dev = current_device();
   if (dev < 0) return SDATTN_ERR_CUDA;
-  auto kern = sdattn::flash_kernel<D, NQ, BN, BF16, NPOLY>;
+  auto kern = sdattn::flash_kernel<D, NQ, BN, BF16, NPOLY, PREC>;
   static std::atomic<uint64_t> smem_done{0};
   if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
 
@@ -439,6 +440,117 @@ sdattn_status dispatch_av(const sdattn_desc* d, const void* A, const float* LS, 
 size_t qk_split_need(const sdattn_desc* d, const QKPlan& pl) {
   const int64_t tiles = static_cast<int64_t>(d->B) * d->H * pl.nrt;
   return pl.nsplit > 1 ? ws_tickets_bytes(d) + static_cast<size_t>(tiles) * 128 * pl.nsplit * sizeof(float2) : 0;
+}
+
+// ---- GroupNorm and gated GELU ----
+// A group is spread over a cluster of up to kGNMaxCluster CTAs, each holding
+// at most kGNThreads x 8 chunks of 8 values.
+constexpr int64_t kGNMaxChunks = int64_t(sdattn::kGNThreads) * 8 * sdattn::kGNMaxCluster;
+
+sdattn_status check_gn(const sdattn_gn_desc* d) {
+  if (!d) return SDATTN_ERR_INVALID_ARG;
+  if (d->B < 1 || d->C < 1 || d->H < 1 || d->W < 1 || d->G < 1 || d->C % d->G != 0) return SDATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(d->eps) || d->eps < 0.f) return SDATTN_ERR_INVALID_ARG;
+  if (d->dtype != SDATTN_F16 && d->dtype != SDATTN_BF16) return SDATTN_ERR_UNSUPPORTED;
+  const int64_t hw = static_cast<int64_t>(d->H) * d->W;
+  const int64_t gsize = hw * (d->C / d->G);
+  if (hw % 8 != 0 || gsize / 8 > kGNMaxChunks) return SDATTN_ERR_UNSUPPORTED;   // also keeps H*W, gsize in int
+  if (static_cast<int64_t>(d->B) * d->C * hw >= (int64_t(1) << 40)) return SDATTN_ERR_UNSUPPORTED;
+  return SDATTN_OK;
+}
+
+// Cluster launch (distributed shared memory between the CTAs of a group),
+// with programmatic stream serialisation like every other launch.
+template <typename... KArgs, typename... Args>
+bool launch_cluster(void (*kern)(KArgs...), int grid, int cluster, int block, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess;
+}
+
+template <int U, bool BF16>
+sdattn_status launch_gn_u(const sdattn::GNParams& p, int64_t groups, int cluster, int threads, cudaStream_t s) {
+  return launch_cluster(sdattn::group_norm_kernel<U, BF16>, static_cast<int>(groups * cluster), cluster, threads, s, p)
+             ? SDATTN_OK
+             : SDATTN_ERR_CUDA;
+}
+
+template <bool BF16>
+sdattn_status launch_gn(const sdattn_gn_desc* d, const void* X, const float* gamma, const float* beta, void* Y,
+                        cudaStream_t s) {
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  const int nsm = sm_count(dev);
+  sdattn::GNParams p;
+  p.X = X;
+  p.Y = Y;
+  p.gamma = gamma;
+  p.beta = beta;
+  p.G = d->G;
+  p.cpg = d->C / d->G;
+  p.HW = d->H * d->W;
+  p.gsize = p.HW * p.cpg;
+  p.eps = d->eps;
+  const int64_t nch = p.gsize / 8;
+  const int64_t groups = static_cast<int64_t>(d->B) * d->G;
+  // Clusters: as few CTAs per group as hold it in registers, more while the
+  // grid would leave SMs idle and each CTA keeps at least a warp of chunks.
+  const int64_t cap = int64_t(sdattn::kGNThreads) * 8;
+  int k = 1;
+  while (k < sdattn::kGNMaxCluster &&
+         ((nch + k - 1) / k > cap || (groups * k < nsm && (nch + 2 * k - 1) / (2 * k) >= 32)))
+    k *= 2;
+  p.cpc = static_cast<int>((nch + k - 1) / k);
+  int u = 1;
+  while (p.cpc > sdattn::kGNThreads * u) u *= 2;
+  const int64_t per = (p.cpc + u - 1) / u;
+  const int threads = static_cast<int>(std::min<int64_t>(sdattn::kGNThreads, std::max<int64_t>(32, (per + 31) / 32 * 32)));
+  switch (u) {
+    case 1: return launch_gn_u<1, BF16>(p, groups, k, threads, s);
+    case 2: return launch_gn_u<2, BF16>(p, groups, k, threads, s);
+    case 4: return launch_gn_u<4, BF16>(p, groups, k, threads, s);
+    case 8: return launch_gn_u<8, BF16>(p, groups, k, threads, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
+}
+
+template <bool BF16>
+sdattn_status launch_geglu(int64_t T, int F, const void* X, void* Y, cudaStream_t s) {
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  sdattn::GegluParams p;
+  p.X = X;
+  p.Y = Y;
+  p.T = T;
+  p.F = F;
+  const int64_t n = T * (F / 8);
+  const int64_t want = (n + 2 * 256 - 1) / (2 * 256);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count(dev)) * 8)));
+  return launch(sdattn::geglu_kernel<BF16>, grid, 256, 0, s, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
+}
+
+// The precise variant: one query tile per CTA, every block of rows whole.
+template <bool BF16>
+sdattn_status dispatch_flash_f32o(const sdattn_desc* d, const void* Q, const void* K, const void* V, float* O,
+                                  float* LS, cudaStream_t s) {
+  switch (d->d) {
+    case 40: return launch_flash<40, 1, 128, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
+    case 80: return launch_flash<80, 1, 128, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
+    case 160: return launch_flash<160, 1, 64, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
 }
 
 template <bool BF16>
@@ -629,6 +741,18 @@ sdattn_status sdattn_flash(const sdattn_desc* desc, const void* Q, const void* K
                                     : dispatch_flash<false>(desc, Q, K, V, O, LS_or_null, ws, s);
 }
 
+sdattn_status sdattn_flash_f32o(const sdattn_desc* desc, const void* Q, const void* K, const void* V, float* O,
+                                float* LS_or_null, void* stream) {
+  const sdattn_status st = check_desc(desc);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !V || !O) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
+  if (LS_or_null && !aligned16(LS_or_null)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return desc->dtype == SDATTN_BF16 ? dispatch_flash_f32o<true>(desc, Q, K, V, O, LS_or_null, s)
+                                    : dispatch_flash_f32o<false>(desc, Q, K, V, O, LS_or_null, s);
+}
+
 sdattn_status sdattn_device_error(uint32_t* detail) {
   if (detail) *detail = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return SDATTN_ERR_CUDA;
@@ -658,6 +782,30 @@ sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc* desc, const void* Q, co
   // The arrival counters must start at zero; the partials are overwritten.
   if (pl.nsplit > 1 && cudaMemsetAsync(ws, 0, ws_tickets_bytes(desc), s) != cudaSuccess) return SDATTN_ERR_CUDA;
   return dispatch_qk<sdattn::kAF32Stats>(desc, Q, K, A, LS, ws, s);
+}
+
+sdattn_status sdattn_group_norm(const sdattn_gn_desc* desc, const void* X, const float* gamma, const float* beta,
+                                void* Y, void* stream) {
+  const sdattn_status st = check_gn(desc);
+  if (st != SDATTN_OK) return st;
+  if (!X || !gamma || !beta || !Y) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(gamma) & 3u) ||
+      (reinterpret_cast<uintptr_t>(beta) & 3u))
+    return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return desc->dtype == SDATTN_BF16 ? launch_gn<true>(desc, X, gamma, beta, Y, s)
+                                    : launch_gn<false>(desc, X, gamma, beta, Y, s);
+}
+
+sdattn_status sdattn_geglu(int64_t T, int32_t F, int32_t dtype, const void* X, void* Y, void* stream) {
+  if (T < 1 || F < 8) return SDATTN_ERR_INVALID_ARG;
+  if (F % 8 != 0) return SDATTN_ERR_UNSUPPORTED;
+  if (dtype != SDATTN_F16 && dtype != SDATTN_BF16) return SDATTN_ERR_UNSUPPORTED;
+  if (T > (int64_t(1) << 40) / F) return SDATTN_ERR_UNSUPPORTED;
+  if (!X || !Y) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dtype == SDATTN_BF16 ? launch_geglu<true>(T, F, X, Y, s) : launch_geglu<false>(T, F, X, Y, s);
 }
 
 const char* sdattn_status_string(sdattn_status status) {

@@ -16,7 +16,7 @@
  *      -> sdattn_qk_stats, sdattn_softmax_av
  *   2. FlashAttention: exact attention computed tile by tile in one kernel
  *      without writing A to memory.
- *      -> sdattn_flash
+ *      -> sdattn_flash (and sdattn_flash_f32o: fp32 O, for bf16 inputs)
  *
  * Variants of the partially fused form, measured against it:
  *   - the page's reduction as a kernel of its own that reads A back
@@ -24,6 +24,11 @@
  *      -> sdattn_qk_scores, sdattn_row_stats, sdattn_softmax_av
  *   - A stored in fp16, halving the bytes of A written and read:
  *      -> sdattn_qk_stats_f16a, sdattn_softmax_av_f16a
+ *
+ * The two specialised kernels the same section names beside attention:
+ * group normalisation in one command, and GELU fused with its split and
+ * multiplication (the UNet's gated feed-forward activation):
+ *      -> sdattn_group_norm, sdattn_geglu
  *
  * The page gives no formula for L and S.  This library reads them as
  *      L_i = max_j A_ij,     S_i = sum_j exp(A_ij - L_i)      (natural base)
@@ -184,6 +189,17 @@ sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K
                            const void *V, void *O, float *LS_or_null, void *ws,
                            size_t ws_bytes, void *stream);
 
+/* FlashAttention form with fp32 output and 16 more bits of P: the same
+ * kernel with one query tile per CTA, where each weight p is carried as its
+ * 16-bit rounding plus the 16-bit rounding of the residual, P V is the sum of
+ * two tensor-core products, and O [B][H][N][d] is written in float32.  This
+ * is the form that holds bf16 inputs to the accuracy bar of fp16 ones (with
+ * 8-bit mantissas, a 16-bit P and a bf16 O would each cost about 1e-3 of
+ * relative error).  Q, K, V: inputs (desc->dtype); O: float32 output;
+ * LS_or_null as for sdattn_flash.  Needs no workspace (no key-range split). */
+sdattn_status sdattn_flash_f32o(const sdattn_desc *desc, const void *Q, const void *K,
+                                const void *V, float *O, float *LS_or_null, void *stream);
+
 /* Allocation-free variant of sdattn_qk_stats.  It has no counterpart in the
  * paper; it exists for callers that cannot allocate device memory (for
  * instance code running under a framework that owns the allocator, or a
@@ -205,6 +221,39 @@ sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K
  *    SDATTN_ERR_WORKSPACE (use sdattn_qk_stats with a caller workspace). */
 sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc *desc, const void *Q, const void *K,
                                       float *A, float *LS, void *stream);
+
+/* Shape of one group normalisation: X and Y are [B][C][H][W] (NCHW,
+ * contiguous), element type dtype; the C channels form G groups of C/G
+ * consecutive channels. */
+typedef struct {
+    int32_t B, C, H, W;   /* batch, channels, height, width */
+    int32_t G;            /* groups; C must be a multiple of G */
+    int32_t dtype;        /* sdattn_dtype of X and Y */
+    float eps;            /* finite, >= 0; added to the variance (1e-6 in SD's UNet) */
+} sdattn_gn_desc;
+
+/* Group normalisation in one launch (summary of the paper, specialised-
+ * kernels paragraphs: channels split into groups, each group normalised on
+ * its own, one GPU command without intermediate tensors).  Each group is
+ * held in registers by a thread-block cluster that combines its partial sums
+ * through distributed shared memory, so x is read once and y written once.  For each batch b
+ * and group g, over the group's (C/G) H W values:
+ *   mean = sum x / n,  var = sum (x - mean)^2 / n   (biased, fp32),
+ *   Y[b][c][h][w] = (X[b][c][h][w] - mean) / sqrt(var + eps) * gamma[c] + beta[c].
+ * X: input; gamma, beta: float32 [C] (4-byte aligned); Y: output (may not
+ * overlap X).  H*W must be a multiple of 8 and a group at most 262144 values;
+ * other shapes return SDATTN_ERR_UNSUPPORTED.  Needs no workspace. */
+sdattn_status sdattn_group_norm(const sdattn_gn_desc *desc, const void *X, const float *gamma,
+                                const float *beta, void *Y, void *stream);
+
+/* The gated GELU of the UNet's feed-forward layers in one launch (summary of
+ * the paper, specialised-kernels paragraphs: GELU's Gaussian error function
+ * fused with the split and multiplication around it).  X [T][2F] is the
+ * projection's output; its first F columns are h, the last F the gate g:
+ *   Y[t][f] = h[t][f] * g/2 * (1 + erf(g / sqrt(2))),   g = X[t][F + f]
+ * (fp32 arithmetic, Y rounded to dtype).  X: input; Y [T][F]: output.
+ * F must be a multiple of 8 (SDATTN_ERR_UNSUPPORTED otherwise), T >= 1. */
+sdattn_status sdattn_geglu(int64_t T, int32_t F, int32_t dtype, const void *X, void *Y, void *stream);
 
 /* Reads and clears this device's error word (synchronises the device).
  * Returns SDATTN_OK, SDATTN_ERR_TIMEOUT, or SDATTN_ERR_CUDA if it cannot be

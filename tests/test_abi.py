@@ -100,6 +100,29 @@ def test_workspace_checked(lib):
     assert lib.sdattn_flash(ctypes.byref(d), ok, ok, ok, ok, None, bad, need, None) == 3
 
 
+def test_group_norm_and_geglu_arguments(lib):
+    from diffusion_unet_attention_b200 import _lib
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    good = _lib.GNDesc(2, 320, 64, 64, 32, 0, 1e-6)
+    for kw, status in [(dict(C=321), 1), (dict(G=0), 1), (dict(B=0), 1), (dict(eps=-1.0), 1),
+                       (dict(eps=float("nan")), 1), (dict(dtype=3), 2), (dict(H=3, W=3), 2),
+                       (dict(C=32 * 65, H=64, W=64), 2)]:
+        f = dict(B=2, C=320, H=64, W=64, G=32, dtype=0, eps=1e-6)
+        f.update(kw)
+        d = _lib.GNDesc(f["B"], f["C"], f["H"], f["W"], f["G"], f["dtype"], f["eps"])
+        assert lib.sdattn_group_norm(ctypes.byref(d), ok, ok, ok, ok, None) == status, kw
+    assert lib.sdattn_group_norm(None, ok, ok, ok, ok, None) == 1
+    assert lib.sdattn_group_norm(ctypes.byref(good), ok, None, ok, ok, None) == 1
+    assert lib.sdattn_group_norm(ctypes.byref(good), bad, ok, ok, ok, None) == 3
+    assert lib.sdattn_geglu(0, 1280, 0, ok, ok, None) == 1
+    assert lib.sdattn_geglu(10, 4, 0, ok, ok, None) == 1
+    assert lib.sdattn_geglu(10, 1284, 0, ok, ok, None) == 2
+    assert lib.sdattn_geglu(10, 1280, 5, ok, ok, None) == 2
+    assert lib.sdattn_geglu(10, 1280, 0, None, ok, None) == 1
+    assert lib.sdattn_geglu(10, 1280, 0, ok, bad, None) == 3
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.sdattn_status_string(s)

@@ -119,3 +119,42 @@ def test_variants_on_64x64_self_sampled():
         del o
     status, detail = sd.device_error()
     assert status == "SDATTN_OK", (status, hex(detail))
+
+
+# ---------------------------------------------------------------------------
+# bf16 under the gate: P carried as two 16-bit parts, O written in fp32
+# ---------------------------------------------------------------------------
+F32O_SHAPES = [(1, 1, 256, 256, 40), (2, 8, 4096, 77, 40), (2, 8, 1024, 1024, 80), (2, 8, 256, 256, 160),
+               (2, 8, 64, 64, 160), (1, 2, 129, 129, 40), (1, 3, 257, 200, 160), (1, 1, 1, 1, 40), (3, 1, 70, 65, 80)]
+
+
+@pytest.mark.parametrize("B,H,N,M,d", F32O_SHAPES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16], ids=["bf16", "f16"])
+def test_flash_f32o_meets_the_gate(B, H, N, M, d, dtype):
+    q, k, v = synth.make_qkv(synth.Shape("p", B, H, N, M, d), 95 + N % 3, call_id=d, dtype=np.float32)
+    tq, tk, tv = (torch.from_numpy(x).to(DEV).to(dtype) for x in (q, k, v))
+    qr, kr, vr = (t.float().cpu().numpy() for t in (tq, tk, tv))     # the values the GPU receives
+    scale = f32(1 / math.sqrt(d))
+    ref = oracle.attention(qr, kr, vr, scale)
+    o, ls = sd.flash_f32o(tq, tk, tv, scale, return_ls=True)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.float32
+    ea, er = gate(o.cpu().numpy(), ref["O"], f"flash_f32o {dtype}")
+    ls_h = ls.cpu().numpy().astype(np.float64)
+    assert np.abs(ls_h[..., 0] - ref["L"]).max() <= L_TOL
+    assert np.abs(ls_h[..., 1] / ref["S"] - 1).max() <= 2e-4    # 16-bit P plus its residual, polynomial exp2
+    print(f"flash_f32o {dtype} {B, H, N, M, d}: max_abs {ea:.3e} rel_frob {er:.3e}")
+
+
+def test_flash_f32o_bf16_64x64_self_sampled():
+    shape = synth.WORKLOADS["self64"]
+    q, k, v = synth.make_qkv(shape, synth.STREAM["self64"], dtype=np.float32)
+    tq, tk, tv = (torch.from_numpy(x).to(DEV).bfloat16() for x in (q, k, v))
+    qr, kr, vr = (t.float().cpu().numpy() for t in (tq, tk, tv))
+    scale = f32(1 / math.sqrt(40))
+    rows = np.unique(np.concatenate([np.arange(0, 4096, 61), np.arange(127, 4096, 128), [4095]]))
+    ref = oracle.attention(qr[:, :, rows], kr, vr, scale)
+    o = sd.flash_f32o(tq, tk, tv, scale)
+    torch.cuda.synchronize()
+    ea, er = gate(o[:, :, torch.from_numpy(rows).to(DEV)].cpu().numpy(), ref["O"], "flash_f32o bf16 64x64")
+    print(f"flash_f32o bf16 64x64 self: max_abs {ea:.3e} rel_frob {er:.3e}")
