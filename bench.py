@@ -61,7 +61,8 @@ def parse_args():
     ap.add_argument("--no-side", action="store_true",
                     help="time the step set only (no per-form, per-kernel or end-to-end extras)")
     ap.add_argument("--case", default=None,
-                    help="FORM:WORKLOAD, e.g. flash:self64 -- run one form on one workload (for profilers)")
+                    help="FORM:WORKLOAD, e.g. flash:self64 -- run one form (flash, qk_stats, softmax_av, partial, "
+                         "or all three kernels) on one workload (for profilers)")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -799,6 +800,10 @@ def run_case(args):
     def once():
         if form == "flash":
             sd.flash(tq, tk, tv, scale, out=o, ws=scratch.ws)
+        elif form == "all":   # the three kernels of the step, one launch each
+            sd.flash(tq, tk, tv, scale, out=o, ws=scratch.ws)
+            sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
+            sd.softmax_av(a, ls, tv, scale, out=o)
         elif form == "qk_stats":
             sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
         elif form == "softmax_av":

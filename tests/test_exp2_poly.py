@@ -52,3 +52,16 @@ def test_matches_exact_powers_of_two_closely():
     x = np.arange(-120, 9, dtype=np.float32)
     y = exp2_poly(x).astype(np.float64)
     assert np.abs(y / np.exp2(x.astype(np.float64)) - 1).max() < 8e-5
+
+
+def test_committed_fit_reproduces_the_kernel_constants():
+    """The coefficients in sm100.cuh are the degree-3 fit of csrc/exp2_poly_fit.py."""
+    import importlib.util
+    path = os.path.join(os.path.dirname(HDR), "exp2_poly_fit.py")
+    spec = importlib.util.spec_from_file_location("exp2_poly_fit", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    c32, lp = mod.fit(3)
+    want, _ = _constants()
+    np.testing.assert_allclose(c32, np.array(want, np.float32), rtol=2e-6, atol=0)
+    assert lp < 7.6e-5 and mod.horner_max_rel(c32) < 8e-5
