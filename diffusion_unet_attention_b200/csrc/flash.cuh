@@ -65,6 +65,11 @@ struct FlashParams {
   int split;
   uint32_t* tickets;   // [G * NQ], all zero on entry and on exit
   float* part;         // [G * NQ][2][ROWF / 4][128 rows][4]: column quads, rows contiguous
+  // Small grids (ksplit > 1, one query tile per CTA): a thread-block cluster
+  // of ksplit CTAs shares unit blockIdx.x / ksplit, CTA `rank` taking key
+  // tiles [rank nkv / ksplit, (rank + 1) nkv / ksplit); the partial rows are
+  // merged across the cluster through distributed shared memory.
+  int ksplit;
 };
 
 // The work of one CTA as a list of segments: key tiles [j0, j1) of unit u.
@@ -78,7 +83,12 @@ struct FlashSegments {
   int u, j0, j1;
   int u_first, j_first, u_last;
   __device__ __forceinline__ explicit FlashSegments(const FlashParams& p) {
-    if (p.split) {
+    if (p.ksplit > 1) {
+      const int rank = static_cast<int>(cluster_rank());
+      u = static_cast<int>(blockIdx.x) / p.ksplit;
+      j0 = rank * p.nkv / p.ksplit;
+      j1 = (rank + 1) * p.nkv / p.ksplit;
+    } else if (p.split) {
       const int64_t w = static_cast<int64_t>(p.units) * p.nkv;
       const int64_t b = w * blockIdx.x / gridDim.x, e = w * (blockIdx.x + 1) / gridDim.x;
       u_first = static_cast<int>(b / p.nkv);
@@ -105,7 +115,9 @@ struct FlashSegments {
   }
   __device__ __forceinline__ bool valid(const FlashParams& p) const { return j0 < j1 && u < p.units; }
   __device__ __forceinline__ void next(const FlashParams& p) {
-    if (p.split) {
+    if (p.ksplit > 1) {
+      u = p.units;   // one segment per CTA
+    } else if (p.split) {
       if (u == u_last) {
         first_whole(p);
       } else {
@@ -166,6 +178,7 @@ struct FlashCfg {
   static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
   static_assert((PREC ? 2 * D : D) % OCW == 0, "whole store passes");
   static_assert(!PREC || NQ == 1, "the precise variant keeps one query tile per CTA");
+  static_assert(NQ > 1 || 128 * (D + 4) * 4 <= STAGES * STAGE, "cluster partial rows fit in the key/value stages");
 };
 
 // A unit whose key range is cut between two CTAs (split schedule) is
@@ -186,6 +199,17 @@ struct FlashCfg {
 // second add, seeing 1).  Exactly one side merges, from the other's rows in
 // the workspace and its own in tensor memory.  With each CTA's head half
 // scheduled first, the tail normally finds the head done.
+// A unit shared by a cluster (ksplit > 1): every CTA leaves, per row r of the
+// tile, its unnormalised O row, running max m (base 2, scaled), row sum l and
+// raw score max in shared memory at the start of its (now idle) key/value
+// stages, rows CPITCH floats apart; after a cluster barrier CTA `rank` merges
+// rows [rank 128 / k, (rank + 1) 128 / k) over the k CTAs in rank order:
+//   m = max m_j,  O = sum_j O_j 2^(m_j - m) / sum_j l_j 2^(m_j - m).
+template <int D>
+struct ClusterRows {
+  static constexpr int CPITCH = D + 4;   // D columns, then (m, l, raw max, 0); 16-byte rows
+};
+
 template <int ROWF>
 __device__ __forceinline__ float4* partial_rows(float* part, int64_t slot, int half) {
   return reinterpret_cast<float4*>(part) + (slot * 2 + half) * (ROWF / 4) * 128;
@@ -659,6 +683,29 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
       uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * EB;
       const int ovalid = p.N - row_w;
       uint8_t* slice = smem + C::OFF_STG + (warp - 4) * RowStage<C::OCW>::BYTES;
+      if constexpr (NQ == 1 && !PREC) {
+        if (p.ksplit > 1) {
+          // this CTA's share of the key range: unnormalised row, m, l, raw max
+          float* prow = reinterpret_cast<float*>(sKV) + r * ClusterRows<D>::CPITCH;
+          float l = 0.f;
+#pragma unroll
+          for (int c8 = 0; c8 <= D / 8; ++c8) {
+            uint32_t o[8];
+            tmem_ld_x8(o_tmem + c8 * 8, o);
+            tmem_wait_ld();
+            reg_fence<8>(o);
+            if (c8 < D / 8) {
+              *reinterpret_cast<uint4*>(prow + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(prow + c8 * 8 + 4) = make_uint4(o[4], o[5], o[6], o[7]);
+            } else {
+              l = __uint_as_float(o[0]);
+            }
+          }
+          *reinterpret_cast<float4*>(prow + D) = make_float4(m_used, l, rawmax, 0.f);
+          tc_fence_before();
+          continue;
+        }
+      }
       if (!(p.split && sg.cut(p))) {
         // O in store passes of PC columns; the first pass also brings the row
         // sum l (column D) when it fits beside them, all behind one wait
@@ -731,6 +778,58 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
   } else {
     // idle warps of the first warp group
     if constexpr (NQ == 2) regs_dec<120>();
+  }
+
+  if constexpr (NQ == 1 && !PREC) {
+    if (p.ksplit > 1) {
+      // every thread of every CTA of the cluster passes both barriers, also
+      // after a wait ran out (the results are then wrong, and the error word says so)
+      constexpr int CP = ClusterRows<D>::CPITCH;
+      const uint32_t k = static_cast<uint32_t>(p.ksplit);
+      const uint32_t rank = cluster_rank();
+      const int u = static_cast<int>(blockIdx.x) / p.ksplit;
+      const int bh = u / p.tph, row0 = (u % p.tph) * 128;
+      __syncwarp();
+      cluster_sync();
+      if (warp >= 4) {
+        const int r0 = static_cast<int>(rank) * 128 / static_cast<int>(k);
+        const int r1 = static_cast<int>(rank + 1) * 128 / static_cast<int>(k);
+        const float* part0 = reinterpret_cast<const float*>(sKV);
+        for (int it = threadIdx.x - 128; it < (r1 - r0) * (D / 8); it += 128) {
+          const int rr = r0 + it / (D / 8), c8 = it % (D / 8);
+          const int row = row0 + rr;
+          if (row >= p.N) continue;
+          float m = -INFINITY;
+          for (uint32_t j = 0; j < k; ++j) m = fmaxf(m, ld_cluster_f32(part0 + rr * CP + D, j));
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float lsum = 0.f, raw = -INFINITY;
+          for (uint32_t j = 0; j < k; ++j) {
+            const float4 st = ld_cluster_f32x4(part0 + rr * CP + D, j);   // (m_j, l_j, raw max_j, 0)
+            const float a = ex2_approx(st.x - m);
+            lsum = fmaf(st.y, a, lsum);
+            raw = fmaxf(raw, st.z);
+            const float4 x0 = ld_cluster_f32x4(part0 + rr * CP + c8 * 8, j);
+            const float4 x1 = ld_cluster_f32x4(part0 + rr * CP + c8 * 8 + 4, j);
+            acc[0] = fmaf(x0.x, a, acc[0]); acc[1] = fmaf(x0.y, a, acc[1]);
+            acc[2] = fmaf(x0.z, a, acc[2]); acc[3] = fmaf(x0.w, a, acc[3]);
+            acc[4] = fmaf(x1.x, a, acc[4]); acc[5] = fmaf(x1.y, a, acc[5]);
+            acc[6] = fmaf(x1.z, a, acc[6]); acc[7] = fmaf(x1.w, a, acc[7]);
+          }
+          const float inv = 1.f / lsum;
+          const int64_t grow = static_cast<int64_t>(bh) * p.N + row;
+          uint4 w;
+          w.x = pack2<BF16>(acc[0] * inv, acc[1] * inv);
+          w.y = pack2<BF16>(acc[2] * inv, acc[3] * inv);
+          w.z = pack2<BF16>(acc[4] * inv, acc[5] * inv);
+          w.w = pack2<BF16>(acc[6] * inv, acc[7] * inv);
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.O) + grow * D * 2 + c8 * 16) = w;
+          if (c8 == 0 && p.LS != nullptr)
+            *reinterpret_cast<float2*>(p.LS + 2 * grow) = make_float2(raw * p.scale, lsum * ex2_approx(m - raw * p.c));
+        }
+      }
+      __syncwarp();
+      cluster_sync();   // no CTA leaves while another may still read its partial rows
+    }
   }
 
   tc_fence_before();

@@ -117,6 +117,28 @@ bool launch(void (*kern)(KArgs...), int grid, int block, int smem, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess;
 }
 
+// Cluster launch (CTAs of a cluster share work through distributed shared
+// memory), with programmatic stream serialisation like every other launch.
+template <typename... KArgs, typename... Args>
+bool launch_cluster(void (*kern)(KArgs...), int grid, int cluster, int block, int smem, cudaStream_t stream,
+                    Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess;
+}
+
 // --------------------------------------------------------------------------
 // Validation
 // --------------------------------------------------------------------------
@@ -330,6 +352,13 @@ sdattn_status launch_av(const sdattn_desc* d, const void* A, const float* LS, co
   p.units = p.BH * p.nrt;
   p.LS = LS;
   p.O = O;
+  // Row tiles filling under half the SMs: a cluster of k CTAs shares each
+  // tile's key blocks (k <= 8, at least one block each, k * tiles <= SMs).
+  int k = 1;
+  if (2 * p.units <= nsm && p.nkb >= 2) k = std::min(std::min(8, p.nkb), nsm / p.units);
+  p.ksplit = k;
+  if (k > 1)
+    return launch_cluster(kern, p.units * k, k, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
   const int grid = p.units < nsm ? p.units : nsm;
   return launch(kern, grid, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
@@ -380,6 +409,16 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   p.split = (ws != nullptr && p.units > nsm && p.nkv >= 2 && eff < 0.9) ? 1 : 0;
   p.tickets = static_cast<uint32_t*>(ws);
   p.part = ws ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flash_ws_tickets_bytes(d, nsm)) : nullptr;
+  // Units filling under half the SMs (one query tile per CTA): a cluster of
+  // k CTAs shares each unit's key tiles (k <= 8, at least one tile each,
+  // k * units <= SMs), merged through distributed shared memory.
+  p.ksplit = 1;
+  if (NQ == 1 && !PREC && 2 * p.units <= nsm && p.nkv >= 2)
+    p.ksplit = std::min(std::min(8, p.nkv), nsm / p.units);
+  if (p.ksplit > 1)
+    return launch_cluster(kern, p.units * p.ksplit, p.ksplit, C::NTHREADS, C::SMEM, stream, mq, mk, mv, mvt, p)
+               ? SDATTN_OK
+               : SDATTN_ERR_CUDA;
   const int grid = p.units < nsm ? p.units : nsm;
   return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, mv, mvt, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
@@ -459,30 +498,9 @@ sdattn_status check_gn(const sdattn_gn_desc* d) {
   return SDATTN_OK;
 }
 
-// Cluster launch (distributed shared memory between the CTAs of a group),
-// with programmatic stream serialisation like every other launch.
-template <typename... KArgs, typename... Args>
-bool launch_cluster(void (*kern)(KArgs...), int grid, int cluster, int block, cudaStream_t stream, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cluster;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess;
-}
-
 template <int U, bool BF16>
 sdattn_status launch_gn_u(const sdattn::GNParams& p, int64_t groups, int cluster, int threads, cudaStream_t s) {
-  return launch_cluster(sdattn::group_norm_kernel<U, BF16>, static_cast<int>(groups * cluster), cluster, threads, s, p)
+  return launch_cluster(sdattn::group_norm_kernel<U, BF16>, static_cast<int>(groups * cluster), cluster, threads, 0, s, p)
              ? SDATTN_OK
              : SDATTN_ERR_CUDA;
 }

@@ -18,6 +18,15 @@
 // The epilogue scales O by 1/S_i and stores it, each warp's 32 consecutive
 // rows through its own shared-memory slice as consecutive 16-byte chunks.
 // Since L_i is final, no rescaling is ever needed.
+//
+// Small grids (row tiles filling under half the SMs): a thread-block cluster
+// of k CTAs shares each row tile, CTA r taking key blocks [r nkb / k,
+// (r + 1) nkb / k).  Since L_i and S_i are final, the k partial products
+// sum_j exp(A_ij - L_i) V_j simply add: each CTA leaves its fp32 partial rows
+// in its own shared memory, and after a cluster barrier CTA r sums rows
+// [r 128 / k, (r + 1) 128 / k) of all k partials (read through distributed
+// shared memory, in rank order, so the result does not depend on timing),
+// scales them by 1/S_i and stores them.
 #pragma once
 
 #include "sm100.cuh"
@@ -29,6 +38,7 @@ struct AVParams {
   int nrt;    // 128-row tiles per (b, h)
   int nkb;    // 64-key blocks
   int units;  // BH * nrt
+  int ksplit; // CTAs of a cluster sharing one row tile's key blocks (1: persistent grid, whole tiles)
   const float* LS;
   void* O;
 };
@@ -46,6 +56,10 @@ struct AVCfg {
   static constexpr int OFF_V = OFF_A + STAGES * A_BYTES;
   static constexpr int OCW = D <= 80 ? D : 80;     // O columns per coalesced store pass
   static constexpr int OFF_STG = OFF_V + STAGES * V_BYTES;   // one store slice per row warp
+  // key split: 128 partial rows of D fp32 (padded: eight lanes writing one
+  // 16-byte chunk of eight rows hit eight bank groups) over the stage buffers
+  static constexpr int PPITCH = D + 4;
+  static_assert(128 * PPITCH * 4 <= OFF_STG, "partial rows fit in the stage buffers");
   static constexpr int OFF_BAR = OFF_STG + 4 * RowStage<OCW>::BYTES;
   static constexpr int NBAR = 4 * STAGES + 4 + 1 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
@@ -113,14 +127,22 @@ __global__ void __launch_bounds__(192, 1)
   grid_dependency_wait();
   grid_launch_dependents();
 
+  // work: whole row tiles over a persistent grid, or (ksplit > 1) one row
+  // tile per cluster, CTA `rank` taking its share of the key blocks
+  const bool split = p.ksplit > 1;
+  const int u_first = split ? static_cast<int>(blockIdx.x) / p.ksplit : static_cast<int>(blockIdx.x);
+  const int u_step = split ? p.units : static_cast<int>(gridDim.x);
+  const int kb0 = split ? static_cast<int>(cluster_rank()) * p.nkb / p.ksplit : 0;
+  const int kb1 = split ? (static_cast<int>(cluster_rank()) + 1) * p.nkb / p.ksplit : p.nkb;
+
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       uint32_t c = 0;
       bool live = true;
-      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
+      for (int u = u_first; u < p.units && live; u += u_step) {
         const int bh = u / p.nrt, rt = u % p.nrt;
-        for (int kb = 0; kb < p.nkb; ++kb, ++c) {
+        for (int kb = kb0; kb < kb1; ++kb, ++c) {
           const uint32_t st = c % C::STAGES, n = c / C::STAGES;
           if (!mbar_wait(&a_empty[st], (n & 1) ^ 1, kSiteAEmpty, abort_flag)) { live = false; break; }
           if (!mbar_wait(&v_empty[st], (n & 1) ^ 1, kSiteVEmpty, abort_flag)) { live = false; break; }
@@ -147,8 +169,8 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t v_base = smem_u32(sV);
       uint32_t c = 0, pc = 0;
       bool live = true;
-      for (int u = blockIdx.x; u < p.units && live; u += gridDim.x) {
-        for (int kb = 0; kb < p.nkb; ++kb, ++c, ++pc) {
+      for (int u = u_first; u < p.units && live; u += u_step) {
+        for (int kb = kb0; kb < kb1; ++kb, ++c, ++pc) {
           const uint32_t st = c % C::STAGES, n = c / C::STAGES;
           const uint32_t pb = pc & 1, np = pc >> 1;
           if (!mbar_wait_warp(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
@@ -159,7 +181,7 @@ __global__ void __launch_bounds__(192, 1)
             // V block, MN-major: 16 keys = two 8-row groups (SBO 1024 B apart);
             // 64-element column slabs C::V_SLAB bytes apart (LBO).
             const uint64_t bd = sdesc_sw128(v_base + st * C::V_BYTES + kk * 2048, C::V_SLAB, 1024);
-            mma_ts(tmem + C::TM_O, tmem + C::TM_P + pb * 32 + kk * 8, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + C::TM_O, tmem + C::TM_P + pb * 32 + kk * 8, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&v_empty[st]);
           mma_commit(&p_empty[pb]);
@@ -178,7 +200,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     uint32_t c = 0, pc = 0, ui = 0;
     bool live = true;
-    for (int u = blockIdx.x; u < p.units && live; u += gridDim.x, ++ui) {
+    for (int u = u_first; u < p.units && live; u += u_step, ++ui) {
       const int bh = u / p.nrt, rt = u % p.nrt;
       const int row = rt * 128 + r;
       float Lr = 0.f, Sr = 1.f;
@@ -188,7 +210,7 @@ __global__ void __launch_bounds__(192, 1)
         Sr = ls.y;
       }
       const float nl = -Lr * L2E;
-      for (int kb = 0; kb < p.nkb; ++kb, ++c, ++pc) {
+      for (int kb = kb0; kb < kb1; ++kb, ++c, ++pc) {
         const uint32_t st = c % C::STAGES, n = c / C::STAGES;
         live = __all_sync(0xffffffffu, mbar_wait(&a_full[st], n & 1, kSiteAFull, abort_flag));
         if (!live) break;
@@ -256,6 +278,22 @@ __global__ void __launch_bounds__(192, 1)
       live = __all_sync(0xffffffffu, mbar_wait(o_full, ui & 1, kSiteOFull, abort_flag));
       if (!live) break;
       tc_fence_after();
+      if (p.ksplit > 1) {
+        // this CTA's share of the key range: unnormalised fp32 rows into shared
+        // memory (the stage buffers are idle now), summed by the cluster below
+        float* prow = reinterpret_cast<float*>(smem) + r * C::PPITCH;
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          uint32_t o[8];
+          tmem_ld_x8(tmem + C::TM_O + c8 * 8 + lane_off, o);
+          tmem_wait_ld();
+          reg_fence<8>(o);
+          *reinterpret_cast<uint4*>(prow + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(prow + c8 * 8 + 4) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        tc_fence_before();
+        continue;
+      }
       const float inv = 1.f / Sr;
       const int row_w = row - lane;   // the warp's first row
       uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * 2;
@@ -281,6 +319,43 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_before();
     }
+  }
+
+  if (p.ksplit > 1) {
+    // every thread of every CTA of the cluster passes both barriers, also
+    // after a wait ran out (the results are then wrong, and the error word says so)
+    const uint32_t k = static_cast<uint32_t>(p.ksplit);
+    const uint32_t rank = cluster_rank();
+    const int bh = u_first / p.nrt, rt = u_first % p.nrt;
+    __syncwarp();
+    cluster_sync();
+    if (warp >= 2) {
+      const int r0 = static_cast<int>(rank) * 128 / static_cast<int>(k);
+      const int r1 = static_cast<int>(rank + 1) * 128 / static_cast<int>(k);
+      const float* part0 = reinterpret_cast<const float*>(smem);
+      for (int it = threadIdx.x - 64; it < (r1 - r0) * (D / 8); it += 128) {
+        const int rr = r0 + it / (D / 8), c8 = it % (D / 8);
+        const int row = rt * 128 + rr;
+        if (row >= p.N) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (uint32_t j = 0; j < k; ++j) {
+          const float4 a = ld_cluster_f32x4(part0 + rr * C::PPITCH + c8 * 8, j);
+          const float4 b = ld_cluster_f32x4(part0 + rr * C::PPITCH + c8 * 8 + 4, j);
+          acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+          acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+        }
+        const int64_t grow = static_cast<int64_t>(bh) * p.N + row;
+        const float inv = 1.f / p.LS[2 * grow + 1];
+        uint4 w;
+        w.x = pack2<BF16>(acc[0] * inv, acc[1] * inv);
+        w.y = pack2<BF16>(acc[2] * inv, acc[3] * inv);
+        w.z = pack2<BF16>(acc[4] * inv, acc[5] * inv);
+        w.w = pack2<BF16>(acc[6] * inv, acc[7] * inv);
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.O) + grow * D * 2 + c8 * 16) = w;
+      }
+    }
+    __syncwarp();
+    cluster_sync();   // no CTA leaves while another may still read its partial rows
   }
 
   tc_fence_before();

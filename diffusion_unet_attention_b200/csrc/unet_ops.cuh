@@ -67,33 +67,6 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
                     pack2<BF16>(f[6], f[7]));
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-
-// All threads of all CTAs of the cluster; shared-memory writes before it are
-// visible to the cluster's reads after it.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Reads a float at the same shared-memory offset as `local`, in cluster CTA `rank`.
-__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
 // Sum over the CTA; every thread gets the total.  `red` holds 32 floats.
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll

@@ -128,7 +128,10 @@ sdattn_status sdattn_qk_stats(const sdattn_desc *desc, const void *Q, const void
  * multiplication by V.
  *   O[b][h][i][c] = (sum_j exp(A_ij - L_i) V[b][h][j][c]) / S_i
  * A, LS (as written by sdattn_qk_stats, or by sdattn_qk_scores followed by
- * sdattn_row_stats), V: inputs; O: output.  Needs no workspace. */
+ * sdattn_row_stats), V: inputs; O: output.  Needs no workspace: when the
+ * 128-row tiles fill under half the SMs, a thread-block cluster of up to 8
+ * CTAs shares each tile's key blocks and adds the partial products through
+ * distributed shared memory in a fixed order. */
 sdattn_status sdattn_softmax_av(const sdattn_desc *desc, const float *A, const float *LS,
                                 const void *V, void *O, void *stream);
 
@@ -184,7 +187,11 @@ sdattn_status sdattn_softmax_av_f16a(const sdattn_desc *desc, const void *A16, c
  * online-softmax merge, in a fixed order, so repeated calls give identical
  * results); this evens out the last wave of work when the row blocks do not
  * divide evenly among the SMs.  Without it every block of rows runs whole in
- * one CTA.  The two schedules agree within rounding. */
+ * one CTA.  The two schedules agree within rounding.  Independently of the
+ * workspace, when the blocks of query rows fill under half the SMs (small
+ * latents, d = 80 and 160), a thread-block cluster of up to 8 CTAs shares
+ * each block's key range and merges the pieces through distributed shared
+ * memory in a fixed order (deterministic results). */
 sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K,
                            const void *V, void *O, float *LS_or_null, void *ws,
                            size_t ws_bytes, void *stream);
