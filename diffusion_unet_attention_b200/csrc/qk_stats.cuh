@@ -20,6 +20,12 @@
 // merged pair to the workspace and bumps an arrival counter; the unit that
 // arrives last merges all splits into LS, then zeroes the partials it read and
 // the counter (no spinning), so a completed call leaves the workspace zero.
+// When every unit has its own CTA and a row tile is split over at most 8 of
+// them (small calls), the splits of a tile form a thread-block cluster
+// instead: each leaves its merged pairs in its shared memory and, after a
+// cluster barrier, CTA `rank` merges rows [rank 128 / k, (rank + 1) 128 / k)
+// of all k splits in split order, read through distributed shared memory;
+// no workspace is used.
 //
 // Store modes (template parameter AMODE):
 //   kAF32Stats  A in fp32 and the row statistics (the partially fused form);
@@ -45,6 +51,7 @@ struct QKParams {
   int cbs;      // column blocks per split
   int units;    // BH * nrt * nsplit
   float scale;
+  int cmerge;         // splits of a row tile merged across a cluster (one unit per CTA)
   float* LS;          // [BH][N][2]
   float2* part;       // [BH * nrt][128][nsplit]
   uint32_t* tickets;  // [BH * nrt]
@@ -64,7 +71,8 @@ struct QKCfg {
   static constexpr int OFF_K = OFF_Q + QBUF * DSLABS * SLAB;
   static constexpr int OFF_STG = OFF_K + KSTAGES * DSLABS * SLAB;
   static constexpr int OFF_MRG = OFF_STG + 4 * EPI * NSTG * STG;   // [2 slots][128 rows] float2
-  static constexpr int OFF_BAR = OFF_MRG + (EPI == 2 ? 2 * 128 * 8 : 0);
+  static constexpr int OFF_CP = OFF_MRG + (EPI == 2 ? 2 * 128 * 8 : 0);   // [128 rows] float2: cluster merge
+  static constexpr int OFF_BAR = OFF_CP + 128 * 8;
   static constexpr int NBAR = 2 * QBUF + 2 * KSTAGES + 4 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;   // + misc words + alignment slack
   static constexpr int NTHREADS = 64 + 128 * EPI;
@@ -343,7 +351,9 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
       }
       // ---- unit result: the merged pair of this split ----
       const int row = rt * 128 + row_local;
-      if (p.nsplit == 1) {
+      if (p.cmerge) {
+        reinterpret_cast<float2*>(smem + C::OFF_CP)[row_local] = make_float2(m_run, s_run);
+      } else if (p.nsplit == 1) {
         if (live && row < p.N)
           *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(m_run, s_run);
       } else {
@@ -376,6 +386,29 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
       }
     }
     if (lane == 0) bulk_wait<0>();
+  }
+
+  if (p.cmerge) {
+    // every thread of every CTA of the cluster passes both barriers, also
+    // after a wait ran out (the results are then wrong, and the error word says so)
+    __syncwarp();
+    cluster_sync();
+    if (warp >= 2 && warp < 6) {   // the first epilogue group merges this CTA's share of the rows
+      int bh, rt, sp, cb0, cb1;
+      qk_decode(p, blockIdx.x, bh, rt, sp, cb0, cb1);
+      const uint32_t k = static_cast<uint32_t>(p.nsplit), rank = cluster_rank();
+      const int r0 = static_cast<int>(rank) * 128 / p.nsplit, r1 = static_cast<int>(rank + 1) * 128 / p.nsplit;
+      const float* cp = reinterpret_cast<const float*>(smem + C::OFF_CP);
+      for (int rr = r0 + static_cast<int>(threadIdx.x) - 64; rr < r1; rr += 128) {
+        const int row = rt * 128 + rr;
+        if (row >= p.N) continue;
+        float m = -INFINITY, sum = 0.f;
+        for (uint32_t j = 0; j < k; ++j) ms_merge(m, sum, ld_cluster_f32(cp + 2 * rr, j), ld_cluster_f32(cp + 2 * rr + 1, j));
+        *reinterpret_cast<float2*>(p.LS + 2 * (static_cast<int64_t>(bh) * p.N + row)) = make_float2(m, sum);
+      }
+    }
+    __syncwarp();
+    cluster_sync();   // no CTA leaves while another may still read its pairs
   }
 
   tc_fence_before();

@@ -33,6 +33,7 @@ using sdattn::RowStatsParams;
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplit = 16;
 constexpr int kMinBlocksPerSplit = 4;
+constexpr int kMinSplitBlocks = 4;   // key tiles per CTA of a cluster-split unit (flash, softmax_av)
 
 // --------------------------------------------------------------------------
 // Driver entry point for tensor-map encoding (no link-time libcuda dependency)
@@ -196,6 +197,10 @@ QKPlan plan_qk(const sdattn_desc* d, int nsm) {
   return pl;
 }
 
+// Small calls (every unit has its own CTA) with at most 8 splits per row tile
+// merge the splits across a thread-block cluster instead of the workspace.
+bool qk_cluster_merge(const QKPlan& pl, int nsm) { return pl.nsplit > 1 && pl.nsplit <= 8 && pl.units <= nsm; }
+
 // Workspace: [tickets: one uint32 per (b, h, row tile), padded to 256 B]
 //            [partials: float2 per (b, h, row tile, row, split)]
 size_t ws_tickets_bytes(const sdattn_desc* d) {
@@ -311,9 +316,13 @@ sdattn_status launch_qk(const sdattn_desc* d, const void* Q, const void* K, void
   p.cbs = pl.cbs;
   p.units = pl.units;
   p.scale = d->scale;
+  p.cmerge = (AMODE != sdattn::kAF32Only && qk_cluster_merge(pl, nsm)) ? 1 : 0;
   p.LS = LS;
   p.tickets = static_cast<uint32_t*>(ws);
   p.part = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + ws_tickets_bytes(d));
+  if (p.cmerge)
+    return launch_cluster(kern, pl.units, pl.nsplit, C::NTHREADS, C::SMEM, stream, mq, mk, ma, p) ? SDATTN_OK
+                                                                                                 : SDATTN_ERR_CUDA;
   const int grid = pl.units < nsm ? pl.units : nsm;
   return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, ma, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
@@ -352,10 +361,14 @@ sdattn_status launch_av(const sdattn_desc* d, const void* A, const float* LS, co
   p.units = p.BH * p.nrt;
   p.LS = LS;
   p.O = O;
-  // Row tiles filling under half the SMs: a cluster of k CTAs shares each
-  // tile's key blocks (k <= 8, at least one block each, k * tiles <= SMs).
+  // Row tiles filling under half the SMs over long key ranges: a cluster of
+  // k CTAs shares each tile's key blocks (k <= 8, k * tiles <= SMs, at least
+  // kMinSplitBlocks blocks each: with fewer, merging the k partial tiles of
+  // d fp32 columns through distributed shared memory costs more than the
+  // blocks it takes off each CTA -- measured on SD's 16x16 calls).
   int k = 1;
-  if (2 * p.units <= nsm && p.nkb >= 2) k = std::min(std::min(8, p.nkb), nsm / p.units);
+  if (2 * p.units <= nsm) k = std::min(std::min(8, p.nkb / kMinSplitBlocks), nsm / p.units);
+  if (k < 2) k = 1;
   p.ksplit = k;
   if (k > 1)
     return launch_cluster(kern, p.units * k, k, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
@@ -409,12 +422,13 @@ sdattn_status launch_flash(const sdattn_desc* d, const void* Q, const void* K, c
   p.split = (ws != nullptr && p.units > nsm && p.nkv >= 2 && eff < 0.9) ? 1 : 0;
   p.tickets = static_cast<uint32_t*>(ws);
   p.part = ws ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + flash_ws_tickets_bytes(d, nsm)) : nullptr;
-  // Units filling under half the SMs (one query tile per CTA): a cluster of
-  // k CTAs shares each unit's key tiles (k <= 8, at least one tile each,
-  // k * units <= SMs), merged through distributed shared memory.
+  // Units filling under half the SMs over long key ranges (one query tile
+  // per CTA): a cluster of k CTAs shares each unit's key tiles (k <= 8,
+  // k * units <= SMs, at least kMinSplitBlocks tiles each, as for softmax_av),
+  // merged through distributed shared memory.
   p.ksplit = 1;
-  if (NQ == 1 && !PREC && 2 * p.units <= nsm && p.nkv >= 2)
-    p.ksplit = std::min(std::min(8, p.nkv), nsm / p.units);
+  if (NQ == 1 && !PREC && 2 * p.units <= nsm) p.ksplit = std::min(std::min(8, p.nkv / kMinSplitBlocks), nsm / p.units);
+  if (p.ksplit < 2) p.ksplit = 1;
   if (p.ksplit > 1)
     return launch_cluster(kern, p.units * p.ksplit, p.ksplit, C::NTHREADS, C::SMEM, stream, mq, mk, mv, mvt, p)
                ? SDATTN_OK
@@ -475,10 +489,11 @@ sdattn_status dispatch_av(const sdattn_desc* d, const void* A, const float* LS, 
 }
 
 // Work split of a qk_stats call with statistics: the scratch that its column
-// split needs (none for a single split).
-size_t qk_split_need(const sdattn_desc* d, const QKPlan& pl) {
+// split needs (none for a single split, or for splits merged in a cluster).
+size_t qk_split_need(const sdattn_desc* d, const QKPlan& pl, int nsm) {
+  if (pl.nsplit == 1 || qk_cluster_merge(pl, nsm)) return 0;
   const int64_t tiles = static_cast<int64_t>(d->B) * d->H * pl.nrt;
-  return pl.nsplit > 1 ? ws_tickets_bytes(d) + static_cast<size_t>(tiles) * 128 * pl.nsplit * sizeof(float2) : 0;
+  return ws_tickets_bytes(d) + static_cast<size_t>(tiles) * 128 * pl.nsplit * sizeof(float2);
 }
 
 // ---- GroupNorm and gated GELU ----
@@ -790,15 +805,16 @@ sdattn_status sdattn_qk_stats_noalloc(const sdattn_desc* desc, const void* Q, co
   if (!aligned16(Q) || !aligned16(K) || !aligned16(A) || !aligned16(LS)) return SDATTN_ERR_ALIGNMENT;
   // Same work split as sdattn_qk_stats; a single split uses no scratch at all.
   const int dev = current_device();
-  const QKPlan pl = plan_qk(desc, sm_count(dev < 0 ? 0 : dev));
-  const size_t need = qk_split_need(desc, pl);
+  const int nsm = sm_count(dev < 0 ? 0 : dev);
+  const QKPlan pl = plan_qk(desc, nsm);
+  const size_t need = qk_split_need(desc, pl, nsm);
   if (need > kNoAllocScratchBytes) return SDATTN_ERR_WORKSPACE;
   if (dev < 0) return SDATTN_ERR_CUDA;
   void* ws = nullptr;
   if (!noalloc_scratch(dev, &ws)) return SDATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The arrival counters must start at zero; the partials are overwritten.
-  if (pl.nsplit > 1 && cudaMemsetAsync(ws, 0, ws_tickets_bytes(desc), s) != cudaSuccess) return SDATTN_ERR_CUDA;
+  if (need > 0 && cudaMemsetAsync(ws, 0, ws_tickets_bytes(desc), s) != cudaSuccess) return SDATTN_ERR_CUDA;
   return dispatch_qk<sdattn::kAF32Stats>(desc, Q, K, A, LS, ws, s);
 }
 

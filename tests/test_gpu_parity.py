@@ -153,6 +153,9 @@ EDGE = [
     (1, 1, 1, 1, 40), (1, 1, 1, 77, 40), (1, 2, 129, 129, 40), (2, 1, 300, 77, 80),
     (1, 1, 64, 64, 160), (1, 3, 257, 200, 160), (2, 2, 130, 1, 80), (1, 1, 128, 2053, 40),
     (1, 1, 383, 1000, 80), (3, 1, 70, 65, 40), (1, 1, 2, 3, 160), (1, 2, 513, 511, 40),
+    # few rows, long key ranges: flash and softmax_av split each block of rows
+    # over a cluster; qk_stats merges 8 column splits through a cluster
+    (2, 8, 256, 4096, 160), (1, 8, 128, 2048, 40), (2, 4, 100, 3000, 80),
 ]
 
 

@@ -219,3 +219,4 @@ def test_gelu_pins_catch_planted_mistakes(mutant):
 def test_geglu_pin_catches_swapped_halves():
     with pytest.raises(AssertionError):
         pin_geglu_split(_geglu_swapped)
+
