@@ -79,11 +79,14 @@ struct FlashParams {
 // With the cut units first, both halves of a cut unit finish early in their
 // CTAs' runs and every CTA ends on a whole unit: the merge of two halves is
 // never the last thing a CTA does.
+// KS: the kernel may run cluster-split units (one query tile per CTA only);
+// the check is compiled out of the two-tile kernel.
+template <bool KS>
 struct FlashSegments {
   int u, j0, j1;
   int u_first, j_first, u_last;
   __device__ __forceinline__ explicit FlashSegments(const FlashParams& p) {
-    if (p.ksplit > 1) {
+    if (KS && p.ksplit > 1) {
       const int rank = static_cast<int>(cluster_rank());
       u = static_cast<int>(blockIdx.x) / p.ksplit;
       j0 = rank * p.nkv / p.ksplit;
@@ -115,7 +118,7 @@ struct FlashSegments {
   }
   __device__ __forceinline__ bool valid(const FlashParams& p) const { return j0 < j1 && u < p.units; }
   __device__ __forceinline__ void next(const FlashParams& p) {
-    if (p.ksplit > 1) {
+    if (KS && p.ksplit > 1) {
       u = p.units;   // one segment per CTA
     } else if (p.split) {
       if (u == u_last) {
@@ -168,6 +171,7 @@ struct FlashCfg {
   static constexpr int MISC = 4 + 4 * NQ;   // words after the barriers
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + MISC * 4 + 1024;
   static constexpr int NTHREADS = 128 + 128 * NQ;
+  static constexpr bool KS = NQ == 1 && !PREC;   // units may be split over a cluster
   // a partial row of a cut unit: D unnormalised O columns, then (m, l, raw max), padded to 16 bytes
   static constexpr int ROWF = (D + 3 + 3) / 4 * 4;
   static_assert(STAGES >= 2, "key/value ring too shallow");
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
     if (lane == 0) {
       uint32_t kvc = 0, nq = 0;
       bool live = true;
-      for (FlashSegments sg(p); sg.valid(p) && live; sg.next(p)) {
+      for (FlashSegments<C::KS> sg(p); sg.valid(p) && live; sg.next(p)) {
         const int bh = sg.u / p.tph, qg = sg.u % p.tph;
         const uint32_t qb = nq % C::QBUF, qn = nq / C::QBUF;
         if (!mbar_wait(&q_empty[qb], (qn & 1) ^ 1, kSiteQEmpty, abort_flag)) { live = false; break; }
@@ -512,7 +516,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
     uint32_t t_base = 0, kv_base = 0, ui = 0;
     bool live = true;
     if (p.inject_stall) live = mbar_wait_warp(stall_bar, 0, kSiteInjected, abort_flag);   // runs out
-    for (FlashSegments sg(p); sg.valid(p) && live; sg.next(p), ++ui) {
+    for (FlashSegments<C::KS> sg(p); sg.valid(p) && live; sg.next(p), ++ui) {
       const uint32_t qb = ui % C::QBUF, qn = ui / C::QBUF;
       if (!mbar_wait_warp(&q_full[qb], qn & 1, kSiteQFull, abort_flag)) { live = false; break; }
       const uint64_t q_desc0 = q_desc00 + ((qb * NQ * C::Q_TILE) >> 4);
@@ -575,7 +579,7 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
     // interleave on the SM instead of contending for the exponential unit.
     if (NQ == 2 && q == 1) live = __all_sync(0xffffffffu, mbar_wait(stagger, 0, kSiteSFull, abort_flag));
     int kcut = 0;          // cut units seen (at most two)
-    for (FlashSegments sg(p); sg.valid(p) && live; sg.next(p)) {
+    for (FlashSegments<C::KS> sg(p); sg.valid(p) && live; sg.next(p)) {
       const int bh = sg.u / p.tph, qg = sg.u % p.tph;
       const int row = (qg * NQ + q) * 128 + r;
       float m_used = -INFINITY, rawmax = -INFINITY;

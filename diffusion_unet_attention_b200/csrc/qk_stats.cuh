@@ -252,92 +252,104 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
         live = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], na & 1, kSiteAccFull, abort_flag));
         if (!live) break;
         tc_fence_after();
-        uint32_t v[128];
-        tmem_ld_x128(tmem + ab * 128 + lane_off, v);
+        const int col0 = cb * 128;
+        const int valid = min(128, p.M - col0);
+        // One half (64 columns) of the block: scale (and round, for fp16 A),
+        // reduce to a partial (m, s) over its valid columns and merge it into
+        // the row's running pair, then stream it to A in 128-byte chunks per
+        // row (32 fp32 or 64 fp16 columns per chunk).
+        auto half = [&](const uint32_t* hv, int h) {
+          float a[64];
+#pragma unroll
+          for (int k = 0; k < 64; ++k) a[k] = __uint_as_float(hv[k]) * p.scale;
+          if constexpr (AMODE == kAF16Stats) {
+            // A is stored in fp16: the statistics are taken from the stored values
+#pragma unroll
+            for (int k = 0; k < 64; k += 2) {
+              const float2 r = __half22float2(__floats2half2_rn(a[k], a[k + 1]));
+              a[k] = r.x;
+              a[k + 1] = r.y;
+            }
+          }
+          const int hvalid = valid - 64 * h;   // valid columns of this half (may be <= 0)
+          if constexpr (AMODE != kAF32Only) {
+            if (hvalid > 0) {
+              // eight independent chains for the max and for the sum, then a tree
+              float mx8[8], sm8[8];
+              if (hvalid >= 64) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = fmax3(a[i], a[8 + i], a[16 + i]);
+#pragma unroll
+                for (int k = 24; k < 64; k += 16)
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], a[k + i], (k + 8 + i < 64) ? a[k + 8 + i] : a[k + i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 64; ++k) mx8[k & 7] = (k < hvalid) ? fmaxf(mx8[k & 7], a[k]) : mx8[k & 7];
+              }
+              const float mb =
+                  fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], fmax3(mx8[5], mx8[6], mx8[7])));
+              const float nmb = -mb * L2E;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
+              if (hvalid >= 64) {
+#pragma unroll
+                for (int k = 0; k < 64; ++k) sm8[k & 7] += ex2_approx(fmaf(a[k], L2E, nmb));
+              } else {
+#pragma unroll
+                for (int k = 0; k < 64; ++k) sm8[k & 7] += (k < hvalid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
+              }
+              const float sb = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+              ms_merge(m_run, s_run, mb, sb);
+            }
+          }
+          constexpr int CC = AMODE == kAF16Stats ? 64 : 32;   // columns per chunk
+#pragma unroll
+          for (int c = 0; c < 64 / CC; ++c) {
+            const int col = col0 + 64 * h + CC * c;
+            if (col >= p.M) break;
+            uint8_t* buf = stg + (sc % C::NSTG) * C::STG;
+            if (lane == 0) bulk_wait_read<C::NSTG - 1>();
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint4 w;
+              if constexpr (AMODE == kAF16Stats) {
+                const float* s8 = a + CC * c + 8 * j;
+                w = make_uint4(pack2<false>(s8[0], s8[1]), pack2<false>(s8[2], s8[3]), pack2<false>(s8[4], s8[5]),
+                               pack2<false>(s8[6], s8[7]));
+              } else {
+                const float* s4 = a + CC * c + 4 * j;
+                w = make_uint4(__float_as_uint(s4[0]), __float_as_uint(s4[1]), __float_as_uint(s4[2]),
+                               __float_as_uint(s4[3]));
+              }
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmA, buf, col, rt * 128 + quarter * 32, bh);
+              bulk_commit();
+            }
+            ++sc;
+          }
+        };
+        // The accumulator in two 64-column loads: the second lands while the
+        // first half is reduced and staged.
+        uint32_t v0[64], v1[64];
+        tmem_ld_x64(tmem + ab * 128 + lane_off, v0);
         tmem_wait_ld();
-        reg_fence<128>(v);
+        reg_fence<64>(v0);
+        tmem_ld_x64(tmem + ab * 128 + 64 + lane_off, v1);
+        half(v0, 0);
+        tmem_wait_ld();
+        reg_fence<64>(v1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
-
-        float a[128];
-#pragma unroll
-        for (int k = 0; k < 128; ++k) a[k] = __uint_as_float(v[k]) * p.scale;
-        if constexpr (AMODE == kAF16Stats) {
-          // A is stored in fp16: the statistics are taken from the stored values
-#pragma unroll
-          for (int k = 0; k < 128; k += 2) {
-            const float2 r = __half22float2(__floats2half2_rn(a[k], a[k + 1]));
-            a[k] = r.x;
-            a[k + 1] = r.y;
-          }
-        }
-        const int col0 = cb * 128;
-        const int valid = min(128, p.M - col0);
-        if constexpr (AMODE != kAF32Only) {
-          // block partial (m_b, s_b) over the valid columns of this 128-column block
-          // eight independent chains for the max and for the sum, then a tree
-          float mx8[8], sm8[8];
-          if (valid == 128) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = fmax3(a[i], a[8 + i], a[16 + i]);
-#pragma unroll
-            for (int k = 24; k < 128; k += 16)
-#pragma unroll
-              for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], a[k + i], (k + 8 + i < 128) ? a[k + 8 + i] : a[k + i]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-            for (int k = 0; k < 128; ++k) mx8[k & 7] = (k < valid) ? fmaxf(mx8[k & 7], a[k]) : mx8[k & 7];
-          }
-          const float mb =
-              fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], fmax3(mx8[5], mx8[6], mx8[7])));
-          const float nmb = -mb * L2E;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
-          if (valid == 128) {
-#pragma unroll
-            for (int k = 0; k < 128; ++k) sm8[k & 7] += ex2_approx(fmaf(a[k], L2E, nmb));
-          } else {
-#pragma unroll
-            for (int k = 0; k < 128; ++k) sm8[k & 7] += (k < valid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
-          }
-          const float sb = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-          ms_merge(m_run, s_run, mb, sb);
-        }
-
-        // stream the block to A: chunks of 128 bytes per row x this warp's 32
-        // rows (32 fp32 or 64 fp16 columns per chunk)
-        constexpr int CC = AMODE == kAF16Stats ? 64 : 32;   // columns per chunk
-#pragma unroll
-        for (int c = 0; c < 128 / CC; ++c) {
-          if (col0 + CC * c >= p.M) break;
-          uint8_t* buf = stg + (sc % C::NSTG) * C::STG;
-          if (lane == 0) bulk_wait_read<C::NSTG - 1>();
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint4 w;
-            if constexpr (AMODE == kAF16Stats) {
-              const float* s8 = a + CC * c + 8 * j;
-              w = make_uint4(pack2<false>(s8[0], s8[1]), pack2<false>(s8[2], s8[3]), pack2<false>(s8[4], s8[5]),
-                             pack2<false>(s8[6], s8[7]));
-            } else {
-              const float* s4 = a + CC * c + 4 * j;
-              w = make_uint4(__float_as_uint(s4[0]), __float_as_uint(s4[1]), __float_as_uint(s4[2]),
-                             __float_as_uint(s4[3]));
-            }
-            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&tmA, buf, col0 + CC * c, rt * 128 + quarter * 32, bh);
-            bulk_commit();
-          }
-          ++sc;
-        }
+        half(v1, 1);
       }
       if constexpr (AMODE == kAF32Only) continue;   // no statistics to finish
       // ---- the two groups' pairs merge; group 0 finishes the unit ----

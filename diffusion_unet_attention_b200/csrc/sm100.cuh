@@ -307,6 +307,18 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld_x64(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : SD_R8(r, 0), SD_R8(r, 8), SD_R8(r, 16), SD_R8(r, 24),
+        SD_R8(r, 32), SD_R8(r, 40), SD_R8(r, 48), SD_R8(r, 56)
+      : "r"(taddr));
+}
+
 // 128 consecutive columns in one load (one TMEM round trip for a 128-key score tile).
 __device__ __forceinline__ void tmem_ld_x128(uint32_t taddr, uint32_t* r) {
   asm volatile(
