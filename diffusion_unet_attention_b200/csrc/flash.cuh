@@ -139,7 +139,10 @@ template <int D, int NQ, int BN, bool PREC = false>
 struct FlashCfg {
   static constexpr int DSLABS = (D + 63) / 64;
   static constexpr int KSTEPS = (D + 15) / 16;
-  static constexpr int PVN = DSLABS * 64;          // P V width: D padded to 64, column D = row sum
+  // P V width: D and the row-sum column D, rounded up to the MMA's multiple of
+  // 16 (48 at d = 40); tensor memory keeps D padded to 64 per query tile
+  static constexpr int PVN = (D + 1 + 15) / 16 * 16;
+  static constexpr int PV_COLS = DSLABS * 64;
   static constexpr int TAIL = D - 64 * (DSLABS - 1);  // V columns loaded into its last slab
   static constexpr int Q_TILE = DSLABS * 128 * 128;
   static constexpr int KV_SLAB = BN * 128;
@@ -156,12 +159,12 @@ struct FlashCfg {
   static constexpr int STAGES_FIT = (232448 - 1024 - 16 - 8 * 32 - QBUF * NQ * Q_TILE - STG_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   // tensor memory per query tile: S (BN fp32), P (BN/2 columns of 16-bit
-  // pairs; with PREC a second such buffer holds P's residual), O (PVN fp32)
+  // pairs; with PREC a second such buffer holds P's residual), O (PV_COLS fp32)
   static constexpr uint32_t TM_S = 0;
   static constexpr uint32_t TM_P = BN;
   static constexpr uint32_t TM_PL = BN + BN / 2;
   static constexpr uint32_t TM_O = BN + (PREC ? BN : BN / 2);
-  static constexpr int QCOLS = TM_O + PVN;
+  static constexpr int QCOLS = TM_O + PV_COLS;
   static constexpr uint32_t TMEM_COLS = NQ * QCOLS <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QBUF * NQ * Q_TILE;
@@ -657,6 +660,16 @@ __global__ void __launch_bounds__(FlashCfg<D, NQ, BN, PREC>::NTHREADS, 1)
               for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
               tmem_st_x16(o_tmem + cc * 32, o);
               tmem_st_x16(o_tmem + cc * 32 + 16, o + 16);
+            }
+            if constexpr (C::PVN % 32 != 0) {
+              constexpr int c0 = C::PVN / 32 * 32;
+              uint32_t o[16];
+              tmem_ld_x16(o_tmem + c0, o);
+              tmem_wait_ld();
+              reg_fence<16>(o);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st_x16(o_tmem + c0, o);
             }
           }
         }
