@@ -250,6 +250,62 @@ def test_flash_64x64_self_split_against_whole():
     assert ea <= 1e-3 and er <= 1e-3
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_flash_two_tile_late_max_raises(dt):
+    """d = 40 with two blocks of 128 query rows per SM or more: the two-tile
+    kernel's lazy max (raised only when a tile's max exceeds the running one
+    by more than 2^8, O rescaled then).  Rows of Q share a direction u with
+    sign +1 (every third warp of rows) or -1; keys 420 and 950 (key tiles 3
+    and 7, the last one ragged) are 1.5 u and 2.5 u, so the +1 rows raise
+    their max twice, late, and end dominated by key 950, while the other
+    warps do not.  Without the row statistics, with them and without the
+    workspace; the split schedule twice, bitwise equal."""
+    H = _sms() + 2
+    N, M = 300, 1000
+    shape = synth.Shape("late max", 1, H, N, M, 40)
+    scale = f32(1 / math.sqrt(40))
+    q, k, v = synth.make_qkv(shape, 85, dtype=np.float32)
+    u = synth.normal(86, (1, H, 1, 40)).astype(np.float32)
+    sign = np.where((np.arange(N) // 32) % 3 == 0, 1.0, -1.0).astype(np.float32)[None, None, :, None]
+    q = 3 * (0.5 * q + sign * u)
+    k[:, :, 420] = 1.5 * u[:, :, 0]
+    k[:, :, 950] = 2.5 * u[:, :, 0]
+    if dt == "f16":
+        tq, tk, tv = to_dev(q.astype(np.float16), k.astype(np.float16), v.astype(np.float16))
+        max_abs, rel = MAX_ABS, REL_FROB
+    else:
+        tq, tk, tv = (t.bfloat16() for t in to_dev(q, k, v))
+        max_abs, rel = 2e-2, 8e-3
+    qh, kh, vh = (t.float().cpu().numpy() for t in (tq, tk, tv))
+    ref = oracle.attention(qh, kh, vh, scale)
+    desc = sd.make_desc(1, H, N, M, 40, tq.dtype, scale)
+    ws = torch.zeros(sd.workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    outs = []
+    for use_ws, want_ls in ((True, False), (True, False), (True, True), (False, False)):
+        obuf, o = guarded((1, H, N, 40), tq.dtype)
+        if want_ls:
+            lsbuf, ls = guarded((1, H, N, 2), torch.float32)
+            sd.flash(tq, tk, tv, scale, out=o, out_ls=ls, ws=ws, use_workspace=use_ws)
+        else:
+            sd.flash(tq, tk, tv, scale, out=o, ws=ws if use_ws else None, use_workspace=use_ws)
+        torch.cuda.synchronize()
+        assert margins_intact(obuf)
+        assert int(torch.count_nonzero(ws)) == 0
+        assert_o(o.float().cpu().numpy(), ref["O"], f"flash {dt} ws={use_ws} ls={want_ls}", max_abs, rel)
+        if want_ls:
+            assert margins_intact(lsbuf)
+            ls_h = ls.cpu().numpy().astype(np.float64)
+            # L is an fp32 sum of exact 16-bit products: its rounding grows with |L|
+            assert np.abs(ls_h[..., 0] - ref["L"]).max() <= L_TOL * (1 + np.abs(ref["L"]).max() / 8)
+            assert np.abs(ls_h[..., 1] / ref["S"] - 1).max() <= (S_RTOL_FLASH if dt == "f16" else 4e-3)
+        outs.append(o.clone())
+    assert torch.equal(outs[0], outs[1])
+    # the data does what it is for: the +1 rows end dominated by key 950
+    w950 = np.exp((qh[0] @ kh[0][:, 950][..., None])[..., 0] * scale - ref["L"][0]) / ref["S"][0]
+    plus = sign[0, 0, :, 0] > 0
+    assert (w950[:, plus] > 0.5).mean() > 0.9 and (w950[:, ~plus] < 1e-3).mean() > 0.9
+
+
 # ---------------------------------------------------------------------------
 # invariants on the GPU outputs
 # ---------------------------------------------------------------------------
