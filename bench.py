@@ -368,6 +368,7 @@ def run_gpu(args, rank, world, local_rank):
         extra = side_measurements(torch, sd, stream, sets, scratch, issue, K=min(K, 50))
         extra["per_call"] = per_call_table(torch, sd, stream, sets, scratch)
         extra["unet_ops"] = unet_ops_table(torch, sd, stream)
+        extra["conv3x3_winograd"] = conv3x3_table(torch, sd, stream)
     if not args.no_side:
         # every rank feeds its own replica from host memory; the job's step is its slowest rank's
         barrier()
@@ -610,6 +611,76 @@ def unet_ops_table(torch, sd, stream, reps=40):
                      "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
         del xs, ys
     return {"note": f"graph of {reps} launches over buffers totalling > 256 MB; fp16", "rows": rows}
+
+
+CONV_SHAPES = [(2, 320, 64, 64), (2, 640, 32, 32), (2, 1280, 16, 16), (2, 1280, 8, 8)]
+
+
+def conv3x3_table(torch, sd, stream, reps=20):
+    """The UNet's 3x3 convolutions (C = K, 512x512 batch 2) by Winograd
+    F(4x4, 3x3) against torch's convolution (cuDNN, an implicit-GEMM library
+    kernel, autotuned), each as a CUDA graph of `reps` calls cycling over
+    inputs and outputs that total more than twice the L2.  The filter is
+    transformed once, outside the timed region (inference reuses it).
+    Effective TFLOP/s counts the direct convolution's 2 * 9 * C * K * N * H * W;
+    the Winograd path's bytes are x read, U read, V written and read, M
+    (fp32) written and read, y written."""
+    peaks, _ = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dev = torch.device("cuda", torch.cuda.current_device())
+    torch.backends.cudnn.benchmark = True
+    rows = []
+
+    def timed(issue, nbuf):
+        for r in range(3):
+            issue(r % nbuf)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    issue(r % nbuf)
+            g.replay()
+            ts = []
+            for _ in range(3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                stream.synchronize()
+                ts.append(a.elapsed_time(b) / reps)
+        del g
+        return statistics.median(ts)
+
+    for (N, C, H, W) in CONV_SHAPES:
+        K = C
+        xbytes = 2 * N * C * H * W
+        nbuf = max(2, math.ceil(256e6 / (2 * xbytes)))
+        gen = torch.Generator(device=dev).manual_seed(C)
+        xs = [torch.randn(N, C, H, W, device=dev, generator=gen).half() for _ in range(nbuf)]
+        ys = [torch.empty(N, K, H, W, device=dev, dtype=torch.float16) for _ in range(nbuf)]
+        w = (torch.randn(K, C, 3, 3, device=dev, generator=gen) / math.sqrt(9 * C)).half()
+        bias = torch.randn(K, device=dev, generator=gen)
+        bias16 = bias.half()
+        U = sd.wino_filter(w)
+        ws = torch.empty(sd.wino_workspace_bytes(N, C, K, H, W), dtype=torch.uint8, device=dev)
+        with torch.cuda.stream(stream):
+            ms_w = timed(lambda i: sd.conv3x3_winograd(xs[i], U, bias, out=ys[i], ws=ws), nbuf)
+            ms_c = timed(lambda i: torch.nn.functional.conv2d(xs[i], w, bias16, padding=1), nbuf)
+        T = N * ((H + 3) // 4) * ((W + 3) // 4)
+        ldm = (T + 3) // 4 * 4
+        path_bytes = xbytes + 36 * K * C * 2 + 2 * 36 * T * C * 2 + 2 * 36 * K * ldm * 4 + 2 * N * K * H * W
+        flops = 2 * 9 * C * K * N * H * W
+        rows.append({"shape": [N, C, H, W], "K": K, "winograd_us": round(ms_w * 1e3, 2), "cudnn_us": round(ms_c * 1e3, 2),
+                     "speedup_vs_cudnn": round(ms_c / ms_w, 2), "direct_gflop": round(flops / 1e9, 2),
+                     "eff_tflops": round(flops / (ms_w * 1e-3) / 1e12, 1),
+                     "cudnn_tflops": round(flops / (ms_c * 1e-3) / 1e12, 1),
+                     "winograd_path_mb": round(path_bytes / 1e6, 1),
+                     "winograd_gbs": round(path_bytes / (ms_w * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(path_bytes / (ms_w * 1e-3) / 1e9 / hbm, 4)})
+        del xs, ys, U, ws
+    return {"note": f"graph of {reps} calls over buffers totalling > 256 MB; fp16, fp32 accumulation; filter "
+                    "transformed once outside the timed region", "rows": rows}
 
 
 def end_to_end(torch, sd, stream, stepset, scratch, steps):

@@ -30,7 +30,8 @@ import torch
 from . import _lib
 
 __all__ = ["qk_stats", "softmax_av", "flash", "flash_f32o", "partially_fused", "qk_scores", "row_stats", "qk_stats_f16a",
-           "softmax_av_f16a", "group_norm", "geglu", "device_error", "a_ld", "a16_ld", "workspace_bytes", "SdattnError", "load_library"]
+           "softmax_av_f16a", "group_norm", "geglu", "wino_filter", "conv3x3_winograd", "wino_workspace_bytes",
+           "device_error", "a_ld", "a16_ld", "workspace_bytes", "SdattnError", "load_library"]
 
 SdattnError = _lib.SdattnError
 load_library = _lib.load
@@ -338,6 +339,64 @@ def geglu(x: torch.Tensor, out: torch.Tensor | None = None):
     st = _lib_handle().sdattn_geglu(T, F, _DTYPES[x.dtype], x.data_ptr(), Y.data_ptr(), _stream(x.device))
     _lib.check("sdattn_geglu", st)
     return Y
+
+
+def _conv_desc(N, C, K, H, W, dtype) -> _lib.ConvDesc:
+    if dtype not in _DTYPES:
+        raise TypeError(f"dtype {dtype} not supported (float16 or bfloat16)")
+    return _lib.ConvDesc(N, C, K, H, W, _DTYPES[dtype])
+
+
+def wino_filter(w: torch.Tensor, out: torch.Tensor | None = None):
+    """Winograd F(4x4, 3x3) filter transform of w [K, C, 3, 3] (fp16 or bf16):
+    U [36, K, C] of w's dtype, computed once per filter."""
+    if w.dim() != 4 or w.shape[2:] != (3, 3) or not w.is_cuda:
+        raise ValueError("w must be a CUDA tensor [K, C, 3, 3]")
+    K, C = w.shape[:2]
+    w = _contig(w)
+    desc = _conv_desc(1, C, K, 4, 4, w.dtype)
+    U = out if out is not None else torch.empty(36, K, C, dtype=w.dtype, device=w.device)
+    if U.shape != (36, K, C) or U.dtype != w.dtype or not U.is_contiguous():
+        raise ValueError("out must be [36, K, C] of w's dtype")
+    st = _lib_handle().sdattn_wino_filter(ctypes.byref(desc), w.data_ptr(), U.data_ptr(), _stream(w.device))
+    _lib.check("sdattn_wino_filter", st)
+    return U
+
+
+def conv3x3_winograd(x: torch.Tensor, U: torch.Tensor, bias: torch.Tensor | None = None,
+                     out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """The UNet's 3x3 convolution (stride 1, zero padding 1) of x [N, C, H, W]
+    with a filter transformed by `wino_filter`, plus an optional fp32 bias [K]:
+    input transform, batched tensor-core product, output transform."""
+    if x.dim() != 4 or not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor [N, C, H, W]")
+    N, C, H, W = x.shape
+    if U.dim() != 3 or U.shape[0] != 36 or U.shape[2] != C or U.dtype != x.dtype:
+        raise ValueError("U must be wino_filter's [36, K, C] of x's dtype")
+    K = U.shape[1]
+    desc = _conv_desc(N, C, K, H, W, x.dtype)
+    need = _lib_handle().sdattn_wino_workspace_bytes(ctypes.byref(desc))
+    if need == 0:
+        raise _lib.SdattnError("sdattn_wino_workspace_bytes", 2)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=x.device)
+    if bias is not None:
+        bias = _contig(bias.to(device=x.device, dtype=torch.float32))
+        if bias.shape != (K,):
+            raise ValueError("bias must be [K]")
+    x, U = _contig(x), _contig(U)
+    Y = out if out is not None else torch.empty(N, K, H, W, dtype=x.dtype, device=x.device)
+    if Y.shape != (N, K, H, W) or Y.dtype != x.dtype or not Y.is_contiguous():
+        raise ValueError("out must be [N, K, H, W] of x's dtype")
+    st = _lib_handle().sdattn_wino_conv3x3(ctypes.byref(desc), x.data_ptr(), U.data_ptr(),
+                                           bias.data_ptr() if bias is not None else None, Y.data_ptr(),
+                                           ws.data_ptr(), ws.numel() * ws.element_size(), _stream(x.device))
+    _lib.check("sdattn_wino_conv3x3", st)
+    return Y
+
+
+def wino_workspace_bytes(N: int, C: int, K: int, H: int, W: int, dtype=torch.float16) -> int:
+    return int(_lib_handle().sdattn_wino_workspace_bytes(ctypes.byref(_conv_desc(N, C, K, H, W, dtype))))
 
 
 def device_error():

@@ -30,6 +30,7 @@ EXPORTS = ("sdattn_a_ld", "sdattn_workspace_bytes", "sdattn_qk_stats", "sdattn_s
            "sdattn_flash_f32o",
            "sdattn_qk_scores", "sdattn_row_stats", "sdattn_a16_ld", "sdattn_qk_stats_f16a",
            "sdattn_softmax_av_f16a", "sdattn_group_norm", "sdattn_geglu", "sdattn_qk_stats_noalloc",
+           "sdattn_wino_filter_bytes", "sdattn_wino_workspace_bytes", "sdattn_wino_filter", "sdattn_wino_conv3x3",
            "sdattn_device_error", "sdattn_status_string", "sdattn_version")
 
 
@@ -43,6 +44,12 @@ class GNDesc(ctypes.Structure):
     """sdattn_gn_desc: shape of one group normalisation."""
     _fields_ = [("B", ctypes.c_int32), ("C", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
                 ("G", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eps", ctypes.c_float)]
+
+
+class ConvDesc(ctypes.Structure):
+    """sdattn_conv_desc: shape of one 3x3 convolution."""
+    _fields_ = [("N", ctypes.c_int32), ("C", ctypes.c_int32), ("K", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("W", ctypes.c_int32), ("dtype", ctypes.c_int32)]
 
 
 class SdattnError(RuntimeError):
@@ -91,6 +98,15 @@ def load(path: str = LIB_PATH):
     lib.sdattn_group_norm.restype = ctypes.c_int
     lib.sdattn_geglu.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
     lib.sdattn_geglu.restype = ctypes.c_int
+    cp = ctypes.POINTER(ConvDesc)
+    lib.sdattn_wino_filter_bytes.argtypes = [cp]
+    lib.sdattn_wino_filter_bytes.restype = sz
+    lib.sdattn_wino_workspace_bytes.argtypes = [cp]
+    lib.sdattn_wino_workspace_bytes.restype = sz
+    lib.sdattn_wino_filter.argtypes = [cp, vp, vp, vp]
+    lib.sdattn_wino_filter.restype = ctypes.c_int
+    lib.sdattn_wino_conv3x3.argtypes = [cp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sdattn_wino_conv3x3.restype = ctypes.c_int
     lib.sdattn_qk_stats_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.sdattn_qk_stats_noalloc.restype = ctypes.c_int
     lib.sdattn_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]

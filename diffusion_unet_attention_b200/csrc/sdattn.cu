@@ -19,6 +19,7 @@
 #include "row_stats.cuh"
 #include "softmax_av.cuh"
 #include "unet_ops.cuh"
+#include "winograd.cuh"
 
 namespace {
 
@@ -574,6 +575,128 @@ sdattn_status launch_geglu(int64_t T, int F, const void* X, void* Y, cudaStream_
   return launch(sdattn::geglu_kernel<BF16>, grid, 256, 0, s, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
+// --------------------------------------------------------------------------
+// Winograd F(4x4, 3x3) convolution (winograd.cuh)
+// --------------------------------------------------------------------------
+sdattn_status check_conv(const sdattn_conv_desc* d) {
+  if (!d) return SDATTN_ERR_INVALID_ARG;
+  if (d->N < 1 || d->C < 1 || d->K < 1 || d->H < 1 || d->W < 1) return SDATTN_ERR_INVALID_ARG;
+  if (d->dtype != SDATTN_F16 && d->dtype != SDATTN_BF16) return SDATTN_ERR_UNSUPPORTED;
+  // C % 8: the transformed rows are whole 16-byte units, as TMA needs;
+  // W <= 4096: one row of input tiles for one channel fits shared memory
+  if (d->C % 8 != 0 || d->W > 4096) return SDATTN_ERR_UNSUPPORTED;
+  const int64_t T = int64_t(d->N) * ((d->H + 3) / 4) * ((d->W + 3) / 4);
+  const int64_t ldm = (T + 3) / 4 * 4;
+  // every index of the 36 planes stays inside 2^31 elements per plane
+  if (T * d->C >= (int64_t(1) << 31) || int64_t(d->K) * ldm >= (int64_t(1) << 31) ||
+      int64_t(d->K) * d->C >= (int64_t(1) << 31) || int64_t(d->N) * d->C * d->H * d->W >= (int64_t(1) << 40))
+    return SDATTN_ERR_UNSUPPORTED;
+  return SDATTN_OK;
+}
+
+sdattn::WinoGeom wino_geom(const sdattn_conv_desc* d, int nsm) {
+  sdattn::WinoGeom g;
+  g.N = d->N;
+  g.C = d->C;
+  g.K = d->K;
+  g.H = d->H;
+  g.W = d->W;
+  g.TH = (d->H + 3) / 4;
+  g.TW = (d->W + 3) / 4;
+  g.T = g.N * g.TH * g.TW;
+  g.ldm = (g.T + 3) / 4 * 4;
+  // channels per input-transform CTA: the six rows of each fit in 96 KB, and
+  // blocks of at least 16 channels are split further while the grid would
+  // give the SMs fewer than four CTAs each (the kernel is latency-bound)
+  const int64_t per_c = int64_t(sdattn::WinoRows::of(g.TW).CS) * 2;
+  g.CB = 64;
+  while (g.CB > 1 && g.CB * per_c > 96 * 1024) g.CB /= 2;
+  while (g.CB > 16 && int64_t(g.N) * g.TH * ((g.C + g.CB - 1) / g.CB) < 4 * int64_t(nsm)) g.CB /= 2;
+  return g;
+}
+
+size_t wino_v_bytes(const sdattn::WinoGeom& g) {
+  return (size_t(36) * g.T * g.C * 2 + 255) / 256 * 256;
+}
+
+size_t wino_ws_bytes(const sdattn::WinoGeom& g) { return wino_v_bytes(g) + size_t(36) * g.K * g.ldm * 4; }
+
+template <bool BF16>
+sdattn_status launch_wino(const sdattn_conv_desc* d, const void* X, const void* U, const float* bias, void* Y,
+                          void* ws, cudaStream_t s) {
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  const int nsm = sm_count(dev);
+  const sdattn::WinoGeom g = wino_geom(d, nsm);
+  uint16_t* V = static_cast<uint16_t*>(ws);
+  float* M = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + wino_v_bytes(g));
+  // input transform
+  {
+    auto kern = sdattn::wino_input_kernel<BF16>;
+    const int smem = g.CB * sdattn::WinoRows::of(g.TW).CS * 2;
+    static std::atomic<uint64_t> smem_done{0};
+    if (!ensure_smem(kern, 96 * 1024, smem_done, dev)) return SDATTN_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(g.N * g.TH), static_cast<unsigned>((g.C + g.CB - 1) / g.CB));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t*>(X), V, g) != cudaSuccess) return SDATTN_ERR_CUDA;
+  }
+  // the 36 products
+  {
+    using C = sdattn::WinoGemmCfg;
+    auto kern = sdattn::wino_gemm_kernel<BF16>;
+    static std::atomic<uint64_t> smem_done{0};
+    if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
+    CUtensorMap mu, mv;
+    const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map_3d(&mu, U, dt, g.C, g.K, 36, uint64_t(g.C) * 2, uint64_t(g.K) * g.C * 2, 64, 128))
+      return SDATTN_ERR_CUDA;
+    if (!make_map_3d(&mv, V, dt, g.C, g.T, 36, uint64_t(g.C) * 2, uint64_t(g.T) * g.C * 2, 64, 128))
+      return SDATTN_ERR_CUDA;
+    CUtensorMap mm;
+    if (!make_map_3d(&mm, M, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.ldm, g.K, 36, uint64_t(g.ldm) * 4,
+                     uint64_t(g.K) * g.ldm * 4, 32, 32))
+      return SDATTN_ERR_CUDA;
+    sdattn::WinoGemmParams p;
+    p.M = M;
+    p.K = g.K;
+    p.T = g.T;
+    p.ldm = g.ldm;
+    p.kbs = (g.K + 127) / 128;
+    p.tbs = (g.T + 127) / 128;
+    p.units = 36 * p.kbs * p.tbs;
+    p.ksteps = (g.C + C::BK - 1) / C::BK;
+    const int grid = p.units < nsm ? p.units : nsm;
+    if (!launch(kern, grid, C::NTHREADS, C::SMEM, s, mu, mv, mm, p)) return SDATTN_ERR_CUDA;
+  }
+  // output transform
+  {
+    const int64_t n = int64_t(g.K) * g.T;
+    const int grid = static_cast<int>((n + 255) / 256);
+    if (!launch(sdattn::wino_output_kernel<BF16>, grid, 256, 0, s, static_cast<const float*>(M), bias,
+                static_cast<uint16_t*>(Y), g))
+      return SDATTN_ERR_CUDA;
+  }
+  return SDATTN_OK;
+}
+
+template <bool BF16>
+sdattn_status launch_wino_filter(const sdattn_conv_desc* d, const void* w, void* U, cudaStream_t s) {
+  const int64_t n = int64_t(d->K) * d->C;
+  const int grid = static_cast<int>((n + 255) / 256);
+  return launch(sdattn::wino_filter_kernel<BF16>, grid, 256, 0, s, static_cast<const uint16_t*>(w),
+                static_cast<uint16_t*>(U), d->K, d->C)
+             ? SDATTN_OK
+             : SDATTN_ERR_CUDA;
+}
+
 // The precise variant: one query tile per CTA, every block of rows whole.
 template <bool BF16>
 sdattn_status dispatch_flash_f32o(const sdattn_desc* d, const void* Q, const void* K, const void* V, float* O,
@@ -840,6 +963,41 @@ sdattn_status sdattn_geglu(int64_t T, int32_t F, int32_t dtype, const void* X, v
   if (!aligned16(X) || !aligned16(Y)) return SDATTN_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return dtype == SDATTN_BF16 ? launch_geglu<true>(T, F, X, Y, s) : launch_geglu<false>(T, F, X, Y, s);
+}
+
+size_t sdattn_wino_filter_bytes(const sdattn_conv_desc* desc) {
+  if (check_conv(desc) != SDATTN_OK) return 0;
+  return size_t(36) * desc->K * desc->C * 2;
+}
+
+size_t sdattn_wino_workspace_bytes(const sdattn_conv_desc* desc) {
+  if (check_conv(desc) != SDATTN_OK) return 0;
+  // the workspace does not depend on the channel blocking
+  return wino_ws_bytes(wino_geom(desc, 148));
+}
+
+sdattn_status sdattn_wino_filter(const sdattn_conv_desc* desc, const void* w, void* U, void* stream) {
+  const sdattn_status st = check_conv(desc);
+  if (st != SDATTN_OK) return st;
+  if (!w || !U) return SDATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(w) & 1u) || !aligned16(U)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return desc->dtype == SDATTN_BF16 ? launch_wino_filter<true>(desc, w, U, s) : launch_wino_filter<false>(desc, w, U, s);
+}
+
+sdattn_status sdattn_wino_conv3x3(const sdattn_conv_desc* desc, const void* X, const void* U, const float* bias,
+                                  void* Y, void* ws, size_t ws_bytes, void* stream) {
+  const sdattn_status st = check_conv(desc);
+  if (st != SDATTN_OK) return st;
+  if (!X || !U || !Y) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(U) || !aligned16(Y) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+    return SDATTN_ERR_ALIGNMENT;
+  const sdattn::WinoGeom g = wino_geom(desc, 148);
+  if (!ws || ws_bytes < wino_ws_bytes(g)) return SDATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return desc->dtype == SDATTN_BF16 ? launch_wino<true>(desc, X, U, bias, Y, ws, s)
+                                    : launch_wino<false>(desc, X, U, bias, Y, ws, s);
 }
 
 const char* sdattn_status_string(sdattn_status status) {

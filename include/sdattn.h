@@ -30,6 +30,10 @@
  * multiplication (the UNet's gated feed-forward activation):
  *      -> sdattn_group_norm, sdattn_geglu
  *
+ * The section's third optimisation, 3x3 convolutions by Winograd's minimal
+ * filtering with 4x4 tiles:
+ *      -> sdattn_wino_filter, sdattn_wino_conv3x3
+ *
  * The page gives no formula for L and S.  This library reads them as
  *      L_i = max_j A_ij,     S_i = sum_j exp(A_ij - L_i)      (natural base)
  * with A = scale * Q K^T, so that softmax(A)_ij = exp(A_ij - L_i) / S_i.
@@ -261,6 +265,43 @@ sdattn_status sdattn_group_norm(const sdattn_gn_desc *desc, const void *X, const
  * (fp32 arithmetic, Y rounded to dtype).  X: input; Y [T][F]: output.
  * F must be a multiple of 8 (SDATTN_ERR_UNSUPPORTED otherwise), T >= 1. */
 sdattn_status sdattn_geglu(int64_t T, int32_t F, int32_t dtype, const void *X, void *Y, void *stream);
+
+/* The UNet's 3x3 convolution by Winograd's minimal filtering (summary of the
+ * paper, Winograd paragraphs: 3x3 convolutions as Winograd convolutions, a
+ * 4x4 tile as the best balance of compute and memory), read as F(4x4, 3x3):
+ * 4x4 output tiles from 6x6 input tiles.  Stride 1, zero padding 1 (Y has
+ * X's H x W), cross-correlation as in the UNet, optional bias:
+ *   Y[n][k][h][w] = bias[k] + sum_{c,r,s} Wt[k][c][r][s] X[n][c][h+r-1][w+s-1]
+ * X [N][C][H][W], Wt [K][C][3][3] and Y [N][K][H][W] of element type dtype;
+ * bias float32 [K] or NULL.  C must be a multiple of 8 and W at most 4096
+ * (SDATTN_ERR_UNSUPPORTED otherwise). */
+typedef struct {
+    int32_t N, C, K, H, W;   /* batch, input channels, output channels, height, width; all >= 1 */
+    int32_t dtype;           /* sdattn_dtype of X, Wt, U and Y */
+} sdattn_conv_desc;
+
+/* Bytes of the transformed filter U [36][K][C] (dtype); 0 for an invalid desc. */
+size_t sdattn_wino_filter_bytes(const sdattn_conv_desc *desc);
+
+/* Bytes of the workspace a convolution needs: the transformed input
+ * [36][T][C] (dtype) and the 36 products [36][K][ldm] (float32), T = N
+ * ceil(H/4) ceil(W/4) tiles, ldm = T rounded up to 4.  0 for an invalid desc. */
+size_t sdattn_wino_workspace_bytes(const sdattn_conv_desc *desc);
+
+/* Filter transform, once per filter: U[xi][k][c] = (G Wt[k][c] G^T)[xi] in
+ * fp32, rounded to dtype (G the 6x3 transform of F(4, 3)).  Wt needs 2-byte,
+ * U 16-byte alignment; U holds sdattn_wino_filter_bytes(desc) bytes. */
+sdattn_status sdattn_wino_filter(const sdattn_conv_desc *desc, const void *Wt, void *U, void *stream);
+
+/* The convolution from a transformed filter U: input transform (B^T d B per
+ * tile, fp32, rounded to dtype), a batched tensor-core product over the 36
+ * transformed positions (fp32 accumulation), output transform (A^T m A, fp32)
+ * plus bias, rounded to dtype: three launches on `stream`.  ws: at least
+ * sdattn_wino_workspace_bytes(desc) bytes, 16-byte aligned, caller-owned,
+ * fully overwritten (no state between calls).  X, U, Y 16-byte aligned; bias
+ * 4-byte aligned.  Y may not overlap X, U or ws. */
+sdattn_status sdattn_wino_conv3x3(const sdattn_conv_desc *desc, const void *X, const void *U, const float *bias,
+                                  void *Y, void *ws, size_t ws_bytes, void *stream);
 
 /* Reads and clears this device's error word (synchronises the device).
  * Returns SDATTN_OK, SDATTN_ERR_TIMEOUT, or SDATTN_ERR_CUDA if it cannot be

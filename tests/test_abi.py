@@ -123,6 +123,38 @@ def test_group_norm_and_geglu_arguments(lib):
     assert lib.sdattn_geglu(10, 1280, 0, ok, bad, None) == 3
 
 
+def test_winograd_arguments(lib):
+    """Shape rules, workspace size and argument checks of the Winograd calls,
+    all decided on the host (the pointers below are never dereferenced)."""
+    from diffusion_unet_attention_b200 import _lib
+
+    def cd(N=2, C=320, K=320, H=64, W=64, dtype=0):
+        return ctypes.byref(_lib.ConvDesc(N, C, K, H, W, dtype))
+
+    # U [36][K][C] 16-bit; workspace: V [36][T][C] 16-bit (256-byte rounded) + M [36][K][ldm] fp32
+    assert lib.sdattn_wino_filter_bytes(cd()) == 36 * 320 * 320 * 2
+    T = 2 * 16 * 16
+    assert lib.sdattn_wino_workspace_bytes(cd()) == (36 * T * 320 * 2 + 255) // 256 * 256 + 36 * 320 * T * 4
+    T = 1 * 4 * 3   # 13 x 10 -> 4 x 3 tiles, ldm 12
+    assert lib.sdattn_wino_workspace_bytes(cd(N=1, C=24, K=40, H=13, W=10)) == \
+        (36 * T * 24 * 2 + 255) // 256 * 256 + 36 * 40 * 12 * 4
+    for bad in [dict(C=12), dict(W=4097), dict(dtype=7), dict(N=0), dict(K=0), dict(H=0)]:
+        assert lib.sdattn_wino_filter_bytes(cd(**bad)) == 0, bad
+        assert lib.sdattn_wino_workspace_bytes(cd(**bad)) == 0, bad
+    fake = ctypes.c_void_p(1 << 20)   # 16-byte aligned, never touched
+    need = lib.sdattn_wino_workspace_bytes(cd())
+    conv = lib.sdattn_wino_conv3x3
+    assert conv(cd(), fake, fake, None, fake, fake, need - 1, None) == 4      # workspace too small
+    assert conv(cd(), fake, fake, None, fake, None, need, None) == 4          # no workspace
+    assert conv(cd(C=12), fake, fake, None, fake, fake, need, None) == 2      # C not a multiple of 8
+    assert conv(cd(N=0), fake, fake, None, fake, fake, need, None) == 1
+    assert conv(cd(), ctypes.c_void_p((1 << 20) + 8), fake, None, fake, fake, need, None) == 3
+    assert conv(cd(), fake, fake, ctypes.c_void_p((1 << 20) + 2), fake, fake, need, None) == 3   # bias
+    assert conv(cd(), None, fake, None, fake, fake, need, None) == 1
+    assert lib.sdattn_wino_filter(cd(), fake, ctypes.c_void_p((1 << 20) + 4), None) == 3
+    assert lib.sdattn_wino_filter(cd(C=20), fake, fake, None) == 2
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.sdattn_status_string(s)
