@@ -608,9 +608,9 @@ sdattn::WinoGeom wino_geom(const sdattn_conv_desc* d, int nsm) {
   // channels per input-transform CTA: the six rows of each fit in 96 KB, and
   // blocks of at least 16 channels are split further while the grid would
   // give the SMs fewer than four CTAs each (the kernel is latency-bound)
-  const int64_t per_c = int64_t(sdattn::WinoRows::of(g.TW).CS) * 2;
+  const int64_t per_c = int64_t(sdattn::WinoRows::of(g.TW).PS) * 4 / 2;   // bytes per channel
   g.CB = 64;
-  while (g.CB > 1 && g.CB * per_c > 96 * 1024) g.CB /= 2;
+  while (g.CB > 2 && g.CB * per_c > 96 * 1024) g.CB /= 2;   // an even number: channel pairs
   while (g.CB > 16 && int64_t(g.N) * g.TH * ((g.C + g.CB - 1) / g.CB) < 4 * int64_t(nsm)) g.CB /= 2;
   return g;
 }
@@ -633,12 +633,14 @@ sdattn_status launch_wino(const sdattn_conv_desc* d, const void* X, const void* 
   // input transform
   {
     auto kern = sdattn::wino_input_kernel<BF16>;
-    const int smem = g.CB * sdattn::WinoRows::of(g.TW).CS * 2;
+    const int smem = (g.CB / 2) * sdattn::WinoRows::of(g.TW).PS * 4;
     static std::atomic<uint64_t> smem_done{0};
     if (!ensure_smem(kern, 96 * 1024, smem_done, dev)) return SDATTN_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(g.N * g.TH), static_cast<unsigned>((g.C + g.CB - 1) / g.CB));
-    cfg.blockDim = dim3(256);
+    // one thread per (channel pair, tile) of the CTA's block, 32 to 256
+    const int items = (g.CB / 2) * g.TW;
+    cfg.blockDim = dim3(static_cast<unsigned>(std::min(256, std::max(32, (items + 31) / 32 * 32))));
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

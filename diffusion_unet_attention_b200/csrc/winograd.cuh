@@ -107,110 +107,162 @@ __global__ void __launch_bounds__(256) wino_filter_kernel(const uint16_t* __rest
   for (int xi = 0; xi < 36; ++xi) U[xi * plane + i] = to16<BF16>(u[xi]);
 }
 
-// Shared-memory rows of the input kernel: a channel's six input rows, each
-// holding x's W values from column 8 on (16-byte aligned) and zeros around
-// them (column 7 is w = -1); a channel's block is padded to an odd number of
-// words so that lanes on consecutive channels read distinct banks.
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// wino_bt6 on packed pairs (two channels at once, one f32x2 instruction per step).
+__device__ __forceinline__ void wino_bt6x2(const uint64_t* d, int s, uint64_t* t, int ts) {
+  const uint64_t d0 = d[0], d1 = d[s], d2 = d[2 * s], d3 = d[3 * s], d4 = d[4 * s], d5 = d[5 * s];
+  const uint64_t c4 = f2_pack(4.f, 4.f), cm4 = f2_pack(-4.f, -4.f), cm5 = f2_pack(-5.f, -5.f);
+  const uint64_t c2 = f2_pack(2.f, 2.f);
+  const uint64_t d42 = f2_sub(d4, d2);
+  t[0] = f2_fma(c4, d0, f2_fma(cm5, d2, d4));
+  t[ts] = f2_fma(cm4, f2_add(d1, d2), f2_add(d3, d4));
+  t[2 * ts] = f2_fma(c4, f2_sub(d1, d2), f2_sub(d4, d3));
+  t[3 * ts] = f2_fma(c2, f2_sub(d3, d1), d42);
+  t[4 * ts] = f2_fma(c2, f2_sub(d1, d3), d42);
+  t[5 * ts] = f2_fma(c4, d1, f2_fma(cm5, d3, d5));
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint64_t unpack_pair(uint32_t v) {
+  float2 f;
+  if constexpr (BF16) {
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+  } else {
+    f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+  }
+  return f2_pack(f.x, f.y);
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack_pair(uint64_t v) {
+  float lo, hi;
+  f2_unpack(v, lo, hi);
+  return pack2<BF16>(lo, hi);
+}
+
+// Shared-memory rows of the input kernel, per pair of channels (c, c + 1)
+// interleaved as 32-bit words (low half c): six input rows, each holding x's
+// W columns from word 8 on and zeros around them (word 7 is w = -1); a pair's
+// block is padded to an odd number of words so that lanes on consecutive
+// pairs read distinct banks.
 struct WinoRows {
-  int Wp;   // halves per row: 4 TW + 16, a multiple of 8
-  int CS;   // halves per channel: 6 Wp + 2
+  int Wp;   // words per row: 4 TW + 16
+  int PS;   // words per channel pair: 6 Wp + 1
   __host__ __device__ static WinoRows of(int TW) {
     WinoRows r;
     r.Wp = 4 * TW + 16;
-    r.CS = 6 * r.Wp + 2;
+    r.PS = 6 * r.Wp + 1;
     return r;
   }
 };
 
-// A CTA takes one row of tiles (batch n, tile row th) and CB channels: the
-// six input rows it needs are staged in shared memory with the zero border
-// (16-byte loads, four in flight per thread, when W is a multiple of 8), then
-// each thread transforms (channel, tile) pairs, consecutive threads taking
-// consecutive channels so that V's rows are written contiguously.
+// A CTA takes one row of tiles (batch n, tile row th) and CB channels (an
+// even number): the six input rows of each channel pair are staged in shared
+// memory with the zero border (16-byte loads of both channels' rows, two of
+// each in flight per thread, interleaved into words, when W is a multiple of
+// 8), then each thread transforms one (channel pair, tile) at a time on packed
+// fp32 pairs, consecutive threads taking consecutive pairs so that V's rows
+// are written contiguously, 4 bytes (two channels) per thread.
 template <bool BF16>
 __global__ void __launch_bounds__(256) wino_input_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ V,
                                                          const WinoGeom g) {
-  extern __shared__ __align__(16) uint16_t sx[];   // [CB][CS]
+  extern __shared__ __align__(16) uint32_t sw[];   // [CB / 2][PS]
   const WinoRows L = WinoRows::of(g.TW);
   const int n = blockIdx.x / g.TH, th = blockIdx.x % g.TH;
   const int c0 = blockIdx.y * g.CB;
+  const int P = g.CB / 2;
   grid_dependency_wait();
   grid_launch_dependents();
-  // zeros: columns 0..7 and W+8 .. Wp-1 of every row, and rows outside 0..H-1
-  for (int idx = threadIdx.x; idx < g.CB * 6; idx += blockDim.x) {
-    const int cc = idx / 6, i = idx - cc * 6;
-    uint16_t* row = sx + cc * L.CS + i * L.Wp;
-    const int h = th * 4 - 1 + i, c = c0 + cc;
-    const bool inside = h >= 0 && h < g.H && c < g.C;
-    for (int j = 0; j < L.Wp; ++j)
-      if (!inside || j < 8 || j >= 8 + g.W) row[j] = 0;
+  // zeros: the border words of every row (0..7 and W+8 .. Wp-1), and whole
+  // rows outside 0..H-1 or past the last channel
+  for (int r = threadIdx.x; r < P * 6; r += blockDim.x) {
+    const int pp = r / 6, i = r - pp * 6;
+    const int h = th * 4 - 1 + i, c = c0 + 2 * pp;
+    uint32_t* row = sw + pp * L.PS + i * L.Wp;
+    if (h >= 0 && h < g.H && c < g.C) {
+      for (int j = 0; j < 8; ++j) row[j] = 0u;
+      for (int j = 8 + g.W; j < L.Wp; ++j) row[j] = 0u;
+    } else {
+      for (int j = 0; j < L.Wp; ++j) row[j] = 0u;
+    }
   }
+  const uint16_t* xn = x + static_cast<int64_t>(n) * g.C * g.H * g.W;
   if ((g.W & 7) == 0) {
     const int chunks = g.W / 8;                  // 16-byte pieces per row
-    const int items = g.CB * 6 * chunks;
+    const int items = P * 6 * chunks;
+    for (int base = threadIdx.x; base < items; base += 2 * blockDim.x) {
+      uint4 ra[2], rb[2];
+      int dst[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = base + u * blockDim.x;
+        const int pp = it / (6 * chunks), rem = it - pp * 6 * chunks, i = rem / chunks, ch = rem - i * chunks;
+        const int c = c0 + 2 * pp, h = th * 4 - 1 + i;
+        const bool ok = it < items && c < g.C && h >= 0 && h < g.H;   // C is even: c + 1 < C too
+        dst[u] = ok ? pp * L.PS + i * L.Wp + 8 + ch * 8 : -1;
+        const uint4* ra_p = reinterpret_cast<const uint4*>(xn + (static_cast<int64_t>(c) * g.H + h) * g.W) + ch;
+        const uint4* rb_p = reinterpret_cast<const uint4*>(xn + (static_cast<int64_t>(c + 1) * g.H + h) * g.W) + ch;
+        ra[u] = ok ? __ldcs(ra_p) : make_uint4(0, 0, 0, 0);
+        rb[u] = ok ? __ldcs(rb_p) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (dst[u] < 0) continue;
+        const uint32_t a[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w}, b[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
+        uint32_t* d = sw + dst[u];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          d[2 * k] = __byte_perm(a[k], b[k], 0x5410);       // (c, c+1) of column 2k
+          d[2 * k + 1] = __byte_perm(a[k], b[k], 0x7632);   // (c, c+1) of column 2k + 1
+        }
+      }
+    }
+  } else {
+    const int items = P * 6 * g.W;
     for (int base = threadIdx.x; base < items; base += 4 * blockDim.x) {
-      uint4 r[4];
-      bool ok[4];
+      uint32_t r[4];
       int dst[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int it = base + u * blockDim.x;
-        const int cc = it / (6 * chunks), rem = it - cc * 6 * chunks, i = rem / chunks, ch = rem - i * chunks;
-        const int c = c0 + cc, h = th * 4 - 1 + i;
-        ok[u] = it < items && c < g.C && h >= 0 && h < g.H;
-        dst[u] = cc * L.CS + i * L.Wp + 8 + ch * 8;
-        r[u] = ok[u] ? __ldcs(reinterpret_cast<const uint4*>(x + ((static_cast<int64_t>(n) * g.C + c) * g.H + h) * g.W) + ch)
-                     : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (!ok[u]) continue;
-        // CS is 2 mod 8 halves: a channel's rows start 4-byte aligned, so store as words
-        uint32_t* d32 = reinterpret_cast<uint32_t*>(sx + dst[u]);
-        d32[0] = r[u].x;
-        d32[1] = r[u].y;
-        d32[2] = r[u].z;
-        d32[3] = r[u].w;
-      }
-    }
-  } else {
-    const int items = g.CB * 6 * g.W;
-    for (int base = threadIdx.x; base < items; base += 8 * blockDim.x) {
-      uint16_t r[8];
-      int dst[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int it = base + u * blockDim.x;
-        const int cc = it / (6 * g.W), rem = it - cc * 6 * g.W, i = rem / g.W, wc = rem - i * g.W;
-        const int c = c0 + cc, h = th * 4 - 1 + i;
+        const int pp = it / (6 * g.W), rem = it - pp * 6 * g.W, i = rem / g.W, wc = rem - i * g.W;
+        const int c = c0 + 2 * pp, h = th * 4 - 1 + i;
         const bool ok = it < items && c < g.C && h >= 0 && h < g.H;
-        dst[u] = ok ? cc * L.CS + i * L.Wp + 8 + wc : -1;
-        r[u] = ok ? x[((static_cast<int64_t>(n) * g.C + c) * g.H + h) * g.W + wc] : uint16_t(0);
+        dst[u] = ok ? pp * L.PS + i * L.Wp + 8 + wc : -1;
+        r[u] = ok ? uint32_t(xn[(static_cast<int64_t>(c) * g.H + h) * g.W + wc]) |
+                        (uint32_t(xn[(static_cast<int64_t>(c + 1) * g.H + h) * g.W + wc]) << 16)
+                  : 0u;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (dst[u] >= 0) sx[dst[u]] = r[u];
+      for (int u = 0; u < 4; ++u)
+        if (dst[u] >= 0) sw[dst[u]] = r[u];
     }
   }
   __syncthreads();
   const int64_t plane = static_cast<int64_t>(g.T) * g.C;
-  for (int it = threadIdx.x; it < g.CB * g.TW; it += blockDim.x) {
-    const int cc = it % g.CB, tw = it / g.CB;
-    const int c = c0 + cc;
+  const int64_t tile0 = (static_cast<int64_t>(n) * g.TH + th) * g.TW;
+  for (int it = threadIdx.x; it < P * g.TW; it += blockDim.x) {
+    const int pp = it % P, tw = it / P;
+    const int c = c0 + 2 * pp;
     if (c >= g.C) continue;
-    float d[36], t[36], v[36];
-    const uint16_t* src = sx + cc * L.CS + 7 + tw * 4;   // column 7 is w = -1
+    uint64_t d[36], t[36];
+    const uint32_t* src = sw + pp * L.PS + 7 + tw * 4;   // word 7 is w = -1
 #pragma unroll
     for (int i = 0; i < 6; ++i)
 #pragma unroll
-      for (int j = 0; j < 6; ++j) d[6 * i + j] = ld16<BF16>(src + i * L.Wp + j);
+      for (int j = 0; j < 6; ++j) d[6 * i + j] = unpack_pair<BF16>(src[i * L.Wp + j]);
 #pragma unroll
-    for (int col = 0; col < 6; ++col) wino_bt6(d + col, 6, t + col, 6);     // t = B^T d
+    for (int col = 0; col < 6; ++col) wino_bt6x2(d + col, 6, t + col, 6);     // t = B^T d
 #pragma unroll
-    for (int row = 0; row < 6; ++row) wino_bt6(t + 6 * row, 1, v + 6 * row, 1);   // v = t B
-    const int64_t tile = (static_cast<int64_t>(n) * g.TH + th) * g.TW + tw;
+    for (int row = 0; row < 6; ++row) wino_bt6x2(t + 6 * row, 1, d + 6 * row, 1);   // v = t B (into d)
+    uint32_t* out = reinterpret_cast<uint32_t*>(V + (tile0 + tw) * g.C + c);
 #pragma unroll
-    for (int xi = 0; xi < 36; ++xi) V[xi * plane + tile * g.C + c] = to16<BF16>(v[xi]);
+    for (int xi = 0; xi < 36; ++xi) out[xi * (plane / 2)] = pack_pair<BF16>(d[xi]);
   }
 }
 
