@@ -54,17 +54,6 @@ __device__ __forceinline__ uint16_t to16(float f) {
   }
 }
 
-// t = B^T d for one column of a 6x6 input tile (stride s between its entries).
-__device__ __forceinline__ void wino_bt6(const float* d, int s, float* t, int ts) {
-  const float d0 = d[0], d1 = d[s], d2 = d[2 * s], d3 = d[3 * s], d4 = d[4 * s], d5 = d[5 * s];
-  t[0] = fmaf(4.f, d0, fmaf(-5.f, d2, d4));
-  t[ts] = fmaf(-4.f, d1 + d2, d3 + d4);
-  t[2 * ts] = fmaf(4.f, d1 - d2, d4 - d3);
-  t[3 * ts] = fmaf(2.f, d3 - d1, d4 - d2);
-  t[4 * ts] = fmaf(2.f, d1 - d3, d4 - d2);
-  t[5 * ts] = fmaf(4.f, d1, fmaf(-5.f, d3, d5));
-}
-
 // u = G g for one column of a 3x3 filter (stride s), G the 6x3 filter transform.
 __device__ __forceinline__ void wino_g3(const float* g, int s, float* u, int us) {
   const float g0 = g[0], g1 = g[s], g2 = g[2 * s];
@@ -113,7 +102,9 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   return d;
 }
 
-// wino_bt6 on packed pairs (two channels at once, one f32x2 instruction per step).
+// t = B^T d for one column of a 6x6 input tile (stride s between its entries),
+// B^T the 6x6 input transform, on packed pairs: two channels at once, one
+// f32x2 instruction per step.
 __device__ __forceinline__ void wino_bt6x2(const uint64_t* d, int s, uint64_t* t, int ts) {
   const uint64_t d0 = d[0], d1 = d[s], d2 = d[2 * s], d3 = d[3 * s], d4 = d[4 * s], d5 = d[5 * s];
   const uint64_t c4 = f2_pack(4.f, 4.f), cm4 = f2_pack(-4.f, -4.f), cm5 = f2_pack(-5.f, -5.f);
