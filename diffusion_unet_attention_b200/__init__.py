@@ -29,7 +29,7 @@ import torch
 
 from . import _lib
 
-__all__ = ["qk_stats", "softmax_av", "flash", "flash_f32o", "partially_fused", "qk_scores", "row_stats", "qk_stats_f16a",
+__all__ = ["qk_stats", "softmax_av", "flash", "flash_f32o", "flash_tf32", "partially_fused", "qk_scores", "row_stats", "qk_stats_f16a",
            "softmax_av_f16a", "group_norm", "geglu", "wino_filter", "conv3x3_winograd", "wino_workspace_bytes",
            "device_error", "a_ld", "a16_ld", "workspace_bytes", "SdattnError", "load_library"]
 
@@ -277,6 +277,26 @@ def flash_f32o(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float |
     st = _lib_handle().sdattn_flash_f32o(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), O.data_ptr(),
                                          LS.data_ptr() if LS is not None else None, _stream(q.device))
     _lib.check("sdattn_flash_f32o", st)
+    return (O, LS) if return_ls else O
+
+
+def flash_tf32(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+               out: torch.Tensor | None = None, return_ls: bool = False):
+    """FlashAttention form for fp32 q, k, v [B,H,*,d], read natively (tf32
+    tensor-core products, fp32 sums); returns O [B,H,N,d] float32 (and LS if
+    asked)."""
+    B, H, N, M, d = _check_qk(q, k)
+    if q.dtype != torch.float32 or v.dtype != torch.float32 or v.shape != k.shape or not v.is_cuda:
+        raise TypeError("q, k, v must be float32 CUDA tensors, v shaped like k")
+    q, k, v = _contig(q), _contig(k), _contig(v)
+    desc = _lib.Desc(B, H, N, M, d, _lib.SDATTN_F32, float(_scale(scale, d)))
+    O = out if out is not None else torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if O.shape != (B, H, N, d) or O.dtype != torch.float32 or not O.is_contiguous():
+        raise ValueError("out must be contiguous fp32 [B,H,N,d]")
+    LS = torch.empty((B, H, N, 2), dtype=torch.float32, device=q.device) if return_ls else None
+    st = _lib_handle().sdattn_flash_tf32(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), O.data_ptr(),
+                                         LS.data_ptr() if LS is not None else None, _stream(q.device))
+    _lib.check("sdattn_flash_tf32", st)
     return (O, LS) if return_ls else O
 
 

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libsdattn.so")
 
 SDATTN_F16 = 0
 SDATTN_BF16 = 1
+SDATTN_F32 = 2
 
 STATUS = {
     0: "SDATTN_OK",
@@ -27,7 +28,7 @@ STATUS = {
 
 # Every symbol include/sdattn.h declares.
 EXPORTS = ("sdattn_a_ld", "sdattn_workspace_bytes", "sdattn_qk_stats", "sdattn_softmax_av", "sdattn_flash",
-           "sdattn_flash_f32o",
+           "sdattn_flash_f32o", "sdattn_flash_tf32",
            "sdattn_qk_scores", "sdattn_row_stats", "sdattn_a16_ld", "sdattn_qk_stats_f16a",
            "sdattn_softmax_av_f16a", "sdattn_group_norm", "sdattn_geglu", "sdattn_qk_stats_noalloc",
            "sdattn_wino_filter_bytes", "sdattn_wino_workspace_bytes", "sdattn_wino_filter", "sdattn_wino_conv3x3",
@@ -82,6 +83,8 @@ def load(path: str = LIB_PATH):
     lib.sdattn_softmax_av.restype = ctypes.c_int
     lib.sdattn_flash_f32o.argtypes = [dp, vp, vp, vp, vp, vp, vp]
     lib.sdattn_flash_f32o.restype = ctypes.c_int
+    lib.sdattn_flash_tf32.argtypes = [dp, vp, vp, vp, vp, vp, vp]
+    lib.sdattn_flash_tf32.restype = ctypes.c_int
     lib.sdattn_qk_scores.argtypes = [dp, vp, vp, vp, vp]
     lib.sdattn_qk_scores.restype = ctypes.c_int
     lib.sdattn_row_stats.argtypes = [dp, vp, vp, vp, sz, vp]

@@ -15,6 +15,7 @@
 #include "sdattn.h"
 
 #include "flash.cuh"
+#include "flash_tf32.cuh"
 #include "qk_stats.cuh"
 #include "row_stats.cuh"
 #include "softmax_av.cuh"
@@ -699,6 +700,39 @@ sdattn_status launch_wino_filter(const sdattn_conv_desc* d, const void* w, void*
              : SDATTN_ERR_CUDA;
 }
 
+// fp32 inputs through tf32 products (flash_tf32.cuh): one query tile per CTA.
+template <int D>
+sdattn_status launch_flash_tf32(const sdattn_desc* d, const void* Q, const void* K, const void* V, float* O,
+                                float* LS, cudaStream_t stream) {
+  using C = sdattn::FlashTF32Cfg<D>;
+  const int dev = current_device();
+  if (dev < 0) return SDATTN_ERR_CUDA;
+  auto kern = sdattn::flash_tf32_kernel<D>;
+  static std::atomic<uint64_t> smem_done{0};
+  if (!ensure_smem(kern, C::SMEM, smem_done, dev)) return SDATTN_ERR_CUDA;
+  const int nsm = sm_count(dev);
+  const uint64_t bh = static_cast<uint64_t>(d->B) * d->H;
+  const uint64_t N = d->N, M = d->M;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_3d(&mq, Q, f32, D, N, bh, D * 4, N * D * 4, 32, 128)) return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&mk, K, f32, D, M, bh, D * 4, M * D * 4, 32, C::BN)) return SDATTN_ERR_CUDA;
+  if (!make_map_3d(&mv, V, f32, D, M, bh, D * 4, M * D * 4, 32, C::BN)) return SDATTN_ERR_CUDA;
+  sdattn::FlashTF32Params p;
+  p.N = d->N;
+  p.M = d->M;
+  p.BH = static_cast<int>(bh);
+  p.tph = (d->N + 127) / 128;
+  p.nkv = (d->M + C::BN - 1) / C::BN;
+  p.units = p.BH * p.tph;
+  p.scale = d->scale;
+  p.c = d->scale * 1.4426950408889634f;
+  p.O = O;
+  p.LS = LS;
+  const int grid = p.units < nsm ? p.units : nsm;
+  return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
+}
+
 // The precise variant: one query tile per CTA, every block of rows whole.
 template <bool BF16>
 sdattn_status dispatch_flash_f32o(const sdattn_desc* d, const void* Q, const void* K, const void* V, float* O,
@@ -909,6 +943,26 @@ sdattn_status sdattn_flash_f32o(const sdattn_desc* desc, const void* Q, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return desc->dtype == SDATTN_BF16 ? dispatch_flash_f32o<true>(desc, Q, K, V, O, LS_or_null, s)
                                     : dispatch_flash_f32o<false>(desc, Q, K, V, O, LS_or_null, s);
+}
+
+sdattn_status sdattn_flash_tf32(const sdattn_desc* desc, const void* Q, const void* K, const void* V, float* O,
+                                float* LS_or_null, void* stream) {
+  if (!desc) return SDATTN_ERR_INVALID_ARG;
+  if (desc->dtype != SDATTN_F32) return SDATTN_ERR_UNSUPPORTED;
+  sdattn_desc d16 = *desc;   // every other rule is the 16-bit entry points'
+  d16.dtype = SDATTN_F16;
+  const sdattn_status st = check_desc(&d16);
+  if (st != SDATTN_OK) return st;
+  if (!Q || !K || !V || !O) return SDATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SDATTN_ERR_ALIGNMENT;
+  if (LS_or_null && !aligned16(LS_or_null)) return SDATTN_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (desc->d) {
+    case 40: return launch_flash_tf32<40>(desc, Q, K, V, O, LS_or_null, s);
+    case 80: return launch_flash_tf32<80>(desc, Q, K, V, O, LS_or_null, s);
+    case 160: return launch_flash_tf32<160>(desc, Q, K, V, O, LS_or_null, s);
+  }
+  return SDATTN_ERR_UNSUPPORTED;
 }
 
 sdattn_status sdattn_device_error(uint32_t* detail) {

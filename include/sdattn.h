@@ -16,7 +16,8 @@
  *      -> sdattn_qk_stats, sdattn_softmax_av
  *   2. FlashAttention: exact attention computed tile by tile in one kernel
  *      without writing A to memory.
- *      -> sdattn_flash (and sdattn_flash_f32o: fp32 O, for bf16 inputs)
+ *      -> sdattn_flash (and sdattn_flash_f32o: fp32 O, for bf16 inputs;
+ *         sdattn_flash_tf32: fp32 inputs, tf32 products, fp32 O)
  *
  * Variants of the partially fused form, measured against it:
  *   - the page's reduction as a kernel of its own that reads A back
@@ -77,7 +78,8 @@ extern "C" {
 
 typedef enum {
     SDATTN_F16 = 0,   /* IEEE binary16 */
-    SDATTN_BF16 = 1   /* bfloat16 */
+    SDATTN_BF16 = 1,  /* bfloat16 */
+    SDATTN_F32 = 2    /* IEEE binary32: sdattn_flash_tf32 only */
 } sdattn_dtype;
 
 /* Shape of one attention call.  scale is applied to Q K^T (1/sqrt(d) in SD). */
@@ -210,6 +212,16 @@ sdattn_status sdattn_flash(const sdattn_desc *desc, const void *Q, const void *K
  * LS_or_null as for sdattn_flash.  Needs no workspace (no key-range split). */
 sdattn_status sdattn_flash_f32o(const sdattn_desc *desc, const void *Q, const void *K,
                                 const void *V, float *O, float *LS_or_null, void *stream);
+
+/* FlashAttention form for fp32 inputs (desc->dtype = SDATTN_F32), without
+ * rounding them to 16 bits first: Q, K, V [B][H][*][d] float32 are read as
+ * fp32 and multiplied on the tensor cores as tf32 (10-bit mantissas); the
+ * weights P are rounded to tf32 (nearest) before P V; every sum is fp32 and
+ * O [B][H][N][d] is written in float32.  LS_or_null as for sdattn_flash.
+ * One 128-row query tile per CTA, no workspace; d in {40, 80, 160}; any
+ * other dtype returns SDATTN_ERR_UNSUPPORTED. */
+sdattn_status sdattn_flash_tf32(const sdattn_desc *desc, const void *Q, const void *K, const void *V,
+                                float *O, float *LS_or_null, void *stream);
 
 /* Allocation-free variant of sdattn_qk_stats.  It has no counterpart in the
  * paper; it exists for callers that cannot allocate device memory (for

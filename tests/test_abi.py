@@ -155,6 +155,20 @@ def test_winograd_arguments(lib):
     assert lib.sdattn_wino_filter(cd(C=20), fake, fake, None) == 2
 
 
+def test_flash_tf32_arguments(lib):
+    """fp32 inputs go only through sdattn_flash_tf32, and it takes only them."""
+    fake = ctypes.c_void_p(1 << 20)
+    f32 = _desc(dtype=2)
+    assert lib.sdattn_flash_tf32(ctypes.byref(_desc(dtype=0)), fake, fake, fake, fake, None, None) == 2
+    assert lib.sdattn_flash_tf32(ctypes.byref(_desc(dtype=2, d=64)), fake, fake, fake, fake, None, None) == 2
+    assert lib.sdattn_flash_tf32(ctypes.byref(f32), fake, None, fake, fake, None, None) == 1
+    assert lib.sdattn_flash_tf32(ctypes.byref(f32), fake, fake, fake, ctypes.c_void_p((1 << 20) + 4), None, None) == 3
+    assert lib.sdattn_flash_tf32(ctypes.byref(_desc(dtype=2, scale=0.0)), fake, fake, fake, fake, None, None) == 1
+    # the 16-bit entry points reject fp32 descriptors
+    assert lib.sdattn_a_ld(ctypes.byref(f32)) == -1
+    assert lib.sdattn_flash(ctypes.byref(f32), fake, fake, fake, fake, None, None, 0, None) == 2
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.sdattn_status_string(s)
