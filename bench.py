@@ -62,7 +62,8 @@ def parse_args():
                     help="time the step set only (no per-form, per-kernel or end-to-end extras)")
     ap.add_argument("--case", default=None,
                     help="FORM:WORKLOAD, e.g. flash:self64 -- run one form (flash, qk_stats, softmax_av, partial, "
-                         "or all three kernels) on one workload (for profilers)")
+                         "or all three kernels) on one workload; or conv3x3:CxH, e.g. conv3x3:320x64 -- one "
+                         "Winograd 3x3 convolution (batch 2, C = K) (for profilers)")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -859,6 +860,9 @@ def run_case(args):
     import torch
     import diffusion_unet_attention_b200 as sd
     form, name = args.case.split(":")
+    if form == "conv3x3":
+        run_conv_case(args, torch, sd, name)
+        return
     call = synth.WORKLOADS[name]
     device = torch.device("cuda", 0)
     q, k, v = synth.make_qkv(call, synth.STREAM[name])
@@ -896,6 +900,39 @@ def run_case(args):
         times.append(e0.elapsed_time(e1) * 1e3)
     status = sd.device_error()
     print(json.dumps({"case": args.case, "shape": call.__dict__, "us": [round(t, 2) for t in times],
+                      "device_error": status[0]}), flush=True)
+    if status[0] != "SDATTN_OK":
+        sys.exit(1)
+
+
+def run_conv_case(args, torch, sd, name):
+    """One of the UNet's 3x3 convolutions (`CxH`: batch 2, C = K channels,
+    H = W) by Winograd: the filter transformed once, then `reps` timed calls
+    after one warm-up, each with CUDA events."""
+    C, H = (int(t) for t in name.split("x"))
+    if (2, C, H, H) not in CONV_SHAPES:
+        raise SystemExit(f"conv3x3 case {name}: not one of the UNet's shapes {CONV_SHAPES}")
+    N, W, K = 2, H, C
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev).manual_seed(C)
+    x = torch.randn(N, C, H, W, device=dev, generator=gen).half()
+    w = (torch.randn(K, C, 3, 3, device=dev, generator=gen) / math.sqrt(9 * C)).half()
+    bias = torch.randn(K, device=dev, generator=gen)
+    U = sd.wino_filter(w)
+    ws = torch.empty(sd.wino_workspace_bytes(N, C, K, H, W), dtype=torch.uint8, device=dev)
+    y = torch.empty(N, K, H, W, device=dev, dtype=torch.float16)
+    sd.conv3x3_winograd(x, U, bias, out=y, ws=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        sd.conv3x3_winograd(x, U, bias, out=y, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    status = sd.device_error()
+    print(json.dumps({"case": args.case, "shape": [N, C, H, W], "K": K, "us": [round(t, 2) for t in times],
                       "device_error": status[0]}), flush=True)
     if status[0] != "SDATTN_OK":
         sys.exit(1)
