@@ -61,8 +61,8 @@ def parse_args():
     ap.add_argument("--no-side", action="store_true",
                     help="time the step set only (no per-form, per-kernel or end-to-end extras)")
     ap.add_argument("--case", default=None,
-                    help="FORM:WORKLOAD, e.g. flash:self64 -- run one form (flash, qk_stats, softmax_av, partial, "
-                         "or all three kernels) on one workload; or conv3x3:CxH, e.g. conv3x3:320x64 -- one "
+                    help="FORM:WORKLOAD, e.g. flash:self64 -- run one form (flash, qk_stats, softmax_av, "
+                         "qk_stats_f16a, softmax_av_f16a, partial, f16a, or all three kernels) on one workload; or conv3x3:CxH, e.g. conv3x3:320x64 -- one "
                          "Winograd 3x3 convolution (batch 2, C = K) (for profilers)")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
@@ -871,6 +871,9 @@ def run_case(args):
     scratch = Scratch(sd, torch, device, [call])
     scale = 1.0 / math.sqrt(call.d)
     a, ls = scratch.views(call)
+    # fp16-stored A: a view of the same scratch, rows of round_up(M, 8) halves
+    lda16 = (call.M + 7) // 8 * 8
+    a16 = scratch.a.view(torch.float16)[:call.B * call.H * call.N * lda16].view(call.B, call.H, call.N, lda16)
 
     def once():
         if form == "flash":
@@ -883,11 +886,20 @@ def run_case(args):
             sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
         elif form == "softmax_av":
             sd.softmax_av(a, ls, tv, scale, out=o)
+        elif form == "qk_stats_f16a":
+            sd.qk_stats_f16a(tq, tk, scale, out_a=a16, out_ls=ls, ws=scratch.ws)
+        elif form == "softmax_av_f16a":
+            sd.softmax_av_f16a(a16, ls, tv, scale, out=o)
+        elif form == "f16a":    # the fp16-A variant's two kernels
+            sd.qk_stats_f16a(tq, tk, scale, out_a=a16, out_ls=ls, ws=scratch.ws)
+            sd.softmax_av_f16a(a16, ls, tv, scale, out=o)
         else:
             scratch.run(call, tq, tk, tv, o, "partial")
 
     if form == "softmax_av":
         sd.qk_stats(tq, tk, scale, out_a=a, out_ls=ls, ws=scratch.ws)
+    elif form == "softmax_av_f16a":
+        sd.qk_stats_f16a(tq, tk, scale, out_a=a16, out_ls=ls, ws=scratch.ws)
     once()
     torch.cuda.synchronize()
     times = []

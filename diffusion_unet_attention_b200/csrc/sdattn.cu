@@ -373,9 +373,9 @@ sdattn_status launch_av(const sdattn_desc* d, const void* A, const float* LS, co
   if (k < 2) k = 1;
   p.ksplit = k;
   if (k > 1)
-    return launch_cluster(kern, p.units * k, k, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
+    return launch_cluster(kern, p.units * k, k, C::NTHREADS, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
   const int grid = p.units < nsm ? p.units : nsm;
-  return launch(kern, grid, 192, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
+  return launch(kern, grid, C::NTHREADS, C::SMEM, stream, ma, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
 template <int D, int NQ, int BN, bool BF16, int NPOLY = 3, bool PREC = false>

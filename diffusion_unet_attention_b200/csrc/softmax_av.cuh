@@ -10,13 +10,20 @@
 // B200 design.  One persistent CTA per SM walks (b*H + h, 128-row tile) units.
 //   warp 0      TMA producer: a ring of (A block 128 x 64, fp32 or fp16, and V
 //               block 64 x d) stages, 128-byte swizzled;
-//   warps 2..5  one query row per thread: reads its 64 scores of the block from
-//               shared memory, computes p = exp(a - L_i) in registers, packs p
-//               to 16 bits and writes it to tensor memory (double-buffered);
+//   warps 2..9  two groups of four row warps, one query row per thread; group
+//               g takes the CTA's key blocks of parity g: reads its 64 scores
+//               of the block from shared memory, computes p = exp(a - L_i) in
+//               registers, packs p to 16 bits and writes it to tensor memory
+//               (P buffer g);
 //   warp 1      tcgen05 MMA issuer: O += P V with P taken from tensor memory
-//               and V from shared memory, O accumulated in tensor memory.
-// The epilogue scales O by 1/S_i and stores it, each warp's 32 consecutive
-// rows through its own shared-memory slice as consecutive 16-byte chunks.
+//               and V from shared memory, O accumulated in tensor memory (two
+//               accumulators, row tiles alternating, so one tile's epilogue
+//               overlaps the next tile's products).
+// Two row warps per scheduler keep the exponentials and the shared-memory
+// reads of one block in flight while the other block's tensor-memory store
+// and hand-offs complete.  Group (tile index & 1) runs a tile's epilogue:
+// it scales O by 1/S_i and stores it, each warp's 32 consecutive rows through
+// its own shared-memory slice as consecutive 16-byte chunks.
 // Since L_i is final, no rescaling is ever needed.
 //
 // Small grids (row tiles filling under half the SMs): a thread-block cluster
@@ -54,24 +61,26 @@ struct AVCfg {
   static constexpr int STAGES = D == 160 ? 3 : 4;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_V = OFF_A + STAGES * A_BYTES;
-  static constexpr int OCW = D <= 80 ? D : 80;     // O columns per coalesced store pass
+  static constexpr int RG = 2;                     // row-warp groups
+  static constexpr int NTHREADS = 64 + 128 * RG;
+  static constexpr int OCW = D <= 80 ? 40 : 80;    // O columns per coalesced store pass
   static constexpr int OFF_STG = OFF_V + STAGES * V_BYTES;   // one store slice per row warp
   // key split: 128 partial rows of D fp32 (padded: eight lanes writing one
   // 16-byte chunk of eight rows hit eight bank groups) over the stage buffers
   static constexpr int PPITCH = D + 4;
   static_assert(128 * PPITCH * 4 <= OFF_STG, "partial rows fit in the stage buffers");
-  static constexpr int OFF_BAR = OFF_STG + 4 * RowStage<OCW>::BYTES;
-  static constexpr int NBAR = 4 * STAGES + 4 + 1 + 1;
+  static constexpr int OFF_BAR = OFF_STG + 4 * RG * RowStage<OCW>::BYTES;
+  static constexpr int NBAR = 4 * STAGES + 4 + 4 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t TM_P = 0;      // two P buffers of 32 columns (128 x 64 16-bit)
-  static constexpr uint32_t TM_O = 64;     // O accumulator, PVN columns
-  static_assert(TM_O + PVN <= TMEM_COLS, "tensor memory budget");
+  static constexpr uint32_t TM_O = 64;     // two O accumulators, PVN columns each
+  static constexpr uint32_t TMEM_COLS = TM_O + 2 * PVN <= 256 ? 256 : 512;
+  static_assert(TM_O + 2 * PVN <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 template <int D, bool BF16, bool AF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
     softmax_av_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
                       const AVParams p) {
   using C = AVCfg<D, AF16>;
@@ -86,8 +95,9 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* v_empty = v_full + C::STAGES;
   uint64_t* p_full = v_empty + C::STAGES;
   uint64_t* p_empty = p_full + 2;
-  uint64_t* o_full = p_empty + 2;
-  uint64_t* drain_bar = o_full + 1;
+  uint64_t* o_full = p_empty + 2;    // [2] per O accumulator
+  uint64_t* o_empty = o_full + 2;    // [2] the accumulator's epilogue has read it
+  uint64_t* drain_bar = o_empty + 2;
   uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
@@ -105,7 +115,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&p_full[i], 4);
       mbar_init(&p_empty[i], 1);
     }
-    mbar_init(o_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 4);
+    }
     mbar_init(drain_bar, 1);
     misc[1] = 0;
     fence_mbar_init();
@@ -167,9 +180,16 @@ __global__ void __launch_bounds__(192, 1)
     {   // the whole warp runs the loop; one elected lane issues
       constexpr uint32_t idesc = idesc_f16(128, C::PVN, BF16, false, true);
       const uint32_t v_base = smem_u32(sV);
-      uint32_t c = 0, pc = 0;
+      uint32_t c = 0, pc = 0, ui = 0;
       bool live = true;
-      for (int u = u_first; u < p.units && live; u += u_step) {
+      for (int u = u_first; u < p.units && live; u += u_step, ++ui) {
+        const uint32_t ob = ui & 1;
+        // the epilogue of tile ui - 2 must have read this accumulator
+        if (ui >= 2 && !mbar_wait_warp(&o_empty[ob], ((ui >> 1) - 1) & 1, kSiteOFull, abort_flag)) {
+          live = false;
+          break;
+        }
+        const uint32_t o_tm = tmem + C::TM_O + ob * C::PVN;
         for (int kb = kb0; kb < kb1; ++kb, ++c, ++pc) {
           const uint32_t st = c % C::STAGES, n = c / C::STAGES;
           const uint32_t pb = pc & 1, np = pc >> 1;
@@ -181,12 +201,12 @@ __global__ void __launch_bounds__(192, 1)
             // V block, MN-major: 16 keys = two 8-row groups (SBO 1024 B apart);
             // 64-element column slabs C::V_SLAB bytes apart (LBO).
             const uint64_t bd = sdesc_sw128(v_base + st * C::V_BYTES + kk * 2048, C::V_SLAB, 1024);
-            mma_ts(tmem + C::TM_O, tmem + C::TM_P + pb * 32 + kk * 8, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            mma_ts(o_tm, tmem + C::TM_P + pb * 32 + kk * 8, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&v_empty[st]);
           mma_commit(&p_empty[pb]);
         }
-        if (live) mma_commit(o_full);
+        if (live) mma_commit(&o_full[ob]);
       }
       volatile uint32_t never = 0;
       mma_commit(drain_bar);
@@ -198,6 +218,7 @@ __global__ void __launch_bounds__(192, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                // row of the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t g = static_cast<uint32_t>(warp - 2) >> 2;   // row group: key blocks c with c % 2 == g
     uint32_t c = 0, pc = 0, ui = 0;
     bool live = true;
     for (int u = u_first; u < p.units && live; u += u_step, ++ui) {
@@ -211,6 +232,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       const float nl = -Lr * L2E;
       for (int kb = kb0; kb < kb1; ++kb, ++c, ++pc) {
+        if ((c & 1) != g) continue;   // the other group's block (P buffer c & 1 is this group's)
         const uint32_t st = c % C::STAGES, n = c / C::STAGES;
         live = __all_sync(0xffffffffu, mbar_wait(&a_full[st], n & 1, kSiteAFull, abort_flag));
         if (!live) break;
@@ -274,8 +296,11 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(&p_full[pb]);
       }
       if (!live) break;
-      // ---- epilogue: O_i / S_i ----
-      live = __all_sync(0xffffffffu, mbar_wait(o_full, ui & 1, kSiteOFull, abort_flag));
+      // ---- epilogue: O_i / S_i, by group ui & 1 ----
+      if ((ui & 1) != g) continue;
+      const uint32_t ob = ui & 1;
+      const uint32_t o_tm = tmem + C::TM_O + ob * C::PVN + lane_off;
+      live = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (ui >> 1) & 1, kSiteOFull, abort_flag));
       if (!live) break;
       tc_fence_after();
       if (p.ksplit > 1) {
@@ -285,26 +310,36 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
           uint32_t o[8];
-          tmem_ld_x8(tmem + C::TM_O + c8 * 8 + lane_off, o);
+          tmem_ld_x8(o_tm + c8 * 8, o);
           tmem_wait_ld();
           reg_fence<8>(o);
           *reinterpret_cast<uint4*>(prow + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(prow + c8 * 8 + 4) = make_uint4(o[4], o[5], o[6], o[7]);
         }
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_empty[ob]);
         continue;
       }
       const float inv = 1.f / Sr;
       const int row_w = row - lane;   // the warp's first row
       uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * 2;
+      // each row warp has a slice of its own: with one key block per tile the
+      // two groups finish alternate tiles at the same time
       uint8_t* slice = smem + C::OFF_STG + (warp - 2) * RowStage<C::OCW>::BYTES;
 #pragma unroll
       for (int pass = 0; pass < D / C::OCW; ++pass) {
         uint32_t o[C::OCW];
 #pragma unroll
-        for (int c8 = 0; c8 < C::OCW / 8; ++c8) tmem_ld_x8(tmem + C::TM_O + pass * C::OCW + c8 * 8 + lane_off, o + c8 * 8);
+        for (int c8 = 0; c8 < C::OCW / 8; ++c8) tmem_ld_x8(o_tm + pass * C::OCW + c8 * 8, o + c8 * 8);
         tmem_wait_ld();
         reg_fence<C::OCW>(o);
+        if (pass == D / C::OCW - 1) {
+          // the accumulator is read: the tile after next may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty[ob]);
+        }
 #pragma unroll
         for (int c8 = 0; c8 < C::OCW / 8; ++c8) {
           const uint32_t* oc = o + c8 * 8;
@@ -333,7 +368,7 @@ __global__ void __launch_bounds__(192, 1)
       const int r0 = static_cast<int>(rank) * 128 / static_cast<int>(k);
       const int r1 = static_cast<int>(rank + 1) * 128 / static_cast<int>(k);
       const float* part0 = reinterpret_cast<const float*>(smem);
-      for (int it = threadIdx.x - 64; it < (r1 - r0) * (D / 8); it += 128) {
+      for (int it = threadIdx.x - 64; it < (r1 - r0) * (D / 8); it += 128 * C::RG) {
         const int rr = r0 + it / (D / 8), c8 = it % (D / 8);
         const int row = rt * 128 + rr;
         if (row >= p.N) continue;
