@@ -259,9 +259,12 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
         // the row's running pair, then stream it to A in 128-byte chunks per
         // row (32 fp32 or 64 fp16 columns per chunk).
         auto half = [&](const uint32_t* hv, int h) {
+          // scale, two columns per instruction (f32x2: each product rounded as alone)
           float a[64];
+          const uint64_t sc2 = f2_pack(p.scale, p.scale);
 #pragma unroll
-          for (int k = 0; k < 64; ++k) a[k] = __uint_as_float(hv[k]) * p.scale;
+          for (int k = 0; k < 64; k += 2)
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(hv[k]), __uint_as_float(hv[k + 1])), sc2), a[k], a[k + 1]);
           if constexpr (AMODE == kAF16Stats) {
             // A is stored in fp16: the statistics are taken from the stored values
 #pragma unroll
@@ -295,8 +298,20 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
 #pragma unroll
               for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
               if (hvalid >= 64) {
+                // column k adds into sum k % 8 in column order, as the scalar
+                // form below, two columns per f32x2 step
+                const uint64_t l2e2 = f2_pack(L2E, L2E), nmb2 = f2_pack(nmb, nmb);
+                uint64_t s2[4];
 #pragma unroll
-                for (int k = 0; k < 64; ++k) sm8[k & 7] += ex2_approx(fmaf(a[k], L2E, nmb));
+                for (int i = 0; i < 4; ++i) s2[i] = f2_pack(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < 64; k += 2) {
+                  float x0, x1;
+                  f2_unpack(f2_fma(f2_pack(a[k], a[k + 1]), l2e2, nmb2), x0, x1);
+                  s2[(k >> 1) & 3] = f2_add(s2[(k >> 1) & 3], f2_pack(ex2_approx(x0), ex2_approx(x1)));
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) f2_unpack(s2[i], sm8[2 * i], sm8[2 * i + 1]);
               } else {
 #pragma unroll
                 for (int k = 0; k < 64; ++k) sm8[k & 7] += (k < hvalid) ? ex2_approx(fmaf(a[k], L2E, nmb)) : 0.f;
@@ -317,7 +332,7 @@ __global__ void __launch_bounds__(QKCfg<D>::NTHREADS, 1)
             for (int j = 0; j < 8; ++j) {
               uint4 w;
               if constexpr (AMODE == kAF16Stats) {
-                const float* s8 = a + CC * c + 8 * j;
+                const float* s8 = a + CC * c + 8 * j;   // already fp16 values: packing is exact
                 w = make_uint4(pack2<false>(s8[0], s8[1]), pack2<false>(s8[2], s8[3]), pack2<false>(s8[4], s8[5]),
                                pack2<false>(s8[6], s8[7]));
               } else {

@@ -10,20 +10,23 @@
 // B200 design.  One persistent CTA per SM walks (b*H + h, 128-row tile) units.
 //   warp 0      TMA producer: a ring of (A block 128 x 64, fp32 or fp16, and V
 //               block 64 x d) stages, 128-byte swizzled;
-//   warps 2..9  two groups of four row warps, one query row per thread; group
-//               g takes the CTA's key blocks of parity g: reads its 64 scores
-//               of the block from shared memory, computes p = exp(a - L_i) in
-//               registers, packs p to 16 bits and writes it to tensor memory
-//               (P buffer g);
+//   warps 2..   RG groups of four row warps, one query row per thread;
+//               group g takes the CTA's key blocks c with c % RG == g: reads
+//               its 64 scores of the block from shared memory, computes
+//               p = exp(a - L_i) in registers, packs p to 16 bits and writes
+//               it to tensor memory (P buffer g);
 //   warp 1      tcgen05 MMA issuer: O += P V with P taken from tensor memory
-//               and V from shared memory, O accumulated in tensor memory (two
-//               accumulators, row tiles alternating, so one tile's epilogue
-//               overlaps the next tile's products).
-// Two row warps per scheduler keep the exponentials and the shared-memory
-// reads of one block in flight while the other block's tensor-memory store
-// and hand-offs complete.  Group (tile index & 1) runs a tile's epilogue:
+//               and V from shared memory, O accumulated in tensor memory
+//               (accumulators rotating over row tiles, so one tile's
+//               epilogue overlaps the next tile's products).
+// Several row warps per scheduler keep the exponentials and shared-memory
+// reads of one block in flight while another block's tensor-memory store
+// and hand-offs complete.  Group (tile index % RG) runs a tile's epilogue:
 // it scales O by 1/S_i and stores it, each warp's 32 consecutive rows through
-// its own shared-memory slice as consecutive 16-byte chunks.
+// its own shared-memory slice as consecutive 16-byte chunks.  Every barrier
+// that a group waits on (its stages of the ring, its P buffer, the O
+// accumulators whose epilogues it runs) is used by that group alone, in
+// order, so no wait can match the parity of an earlier phase.
 // Since L_i is final, no rescaling is ever needed.
 //
 // Small grids (row tiles filling under half the SMs): a thread-block cluster
@@ -58,24 +61,44 @@ struct AVCfg {
   static constexpr int A_BYTES = 128 * BK * (AF16 ? 2 : 4);   // fp32: two 16 KB boxes of 32 columns; fp16: one of 64
   static constexpr int V_SLAB = BK * 128;              // 8 KB: 64 keys x 64 elements
   static constexpr int V_BYTES = DSLABS * V_SLAB;
-  static constexpr int STAGES = D == 160 ? 3 : 4;
+  static constexpr int STAGE_BYTES = A_BYTES + V_BYTES;
+  // Row-warp groups: group g takes the key blocks c with c % RG == g.  The
+  // ring's stage c % STAGES is then refilled for one group only (STAGES is a
+  // multiple of RG), so a group waits on a stage at most one load ahead of
+  // what it consumed there itself.  Were consecutive loads of a stage taken by
+  // different groups, a group could wait for the load after next while the
+  // next is still in flight, and the phase parity it waits for would match
+  // the phase already completed.
+  // The O accumulators rotate over row tiles the same way: tile ui uses
+  // accumulator ui % NOB and group ui % RG runs its epilogue, so NOB is a
+  // multiple of RG and an accumulator's epilogues are always one group's.
+  // Measured at 64x64: with fp32 A two groups keep four stages in flight,
+  // three only three stages (slower); fp16 A fits six stages either way and
+  // gains from the third group (d = 160 has no tensor memory for a third O).
+  static constexpr int RG = (AF16 && D <= 80) ? 3 : 2;
+  static constexpr int NPB = RG == 1 ? 2 : RG;       // P buffers in tensor memory (group g uses buffer g)
+  static constexpr int NOB = RG == 1 ? 2 : RG;       // O accumulators
+  static constexpr int NTHREADS = 64 + 128 * RG;
+  static constexpr int OCW = (D <= 80 || RG > 2) ? 40 : 80;    // O columns per coalesced store pass
+  static constexpr int STG_BYTES = 4 * RG * RowStage<OCW>::BYTES;   // one store slice per row warp
+  static constexpr int FIXED = STG_BYTES + (4 * 6 + 2 * NPB + 2 * NOB + 1) * 8 + 16 + 1024;
+  static constexpr int STAGES_FIT = (232448 - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = (STAGES_FIT < 6 ? STAGES_FIT : 6) / RG * RG;
+  static_assert(STAGES >= 2 && STAGES % RG == 0, "each ring stage serves one row group");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_V = OFF_A + STAGES * A_BYTES;
-  static constexpr int RG = 2;                     // row-warp groups
-  static constexpr int NTHREADS = 64 + 128 * RG;
-  static constexpr int OCW = D <= 80 ? 40 : 80;    // O columns per coalesced store pass
-  static constexpr int OFF_STG = OFF_V + STAGES * V_BYTES;   // one store slice per row warp
+  static constexpr int OFF_STG = OFF_V + STAGES * V_BYTES;
   // key split: 128 partial rows of D fp32 (padded: eight lanes writing one
   // 16-byte chunk of eight rows hit eight bank groups) over the stage buffers
   static constexpr int PPITCH = D + 4;
   static_assert(128 * PPITCH * 4 <= OFF_STG, "partial rows fit in the stage buffers");
-  static constexpr int OFF_BAR = OFF_STG + 4 * RG * RowStage<OCW>::BYTES;
-  static constexpr int NBAR = 4 * STAGES + 4 + 4 + 1;
+  static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
+  static constexpr int NBAR = 4 * STAGES + 2 * NPB + 2 * NOB + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr uint32_t TM_P = 0;      // two P buffers of 32 columns (128 x 64 16-bit)
-  static constexpr uint32_t TM_O = 64;     // two O accumulators, PVN columns each
-  static constexpr uint32_t TMEM_COLS = TM_O + 2 * PVN <= 256 ? 256 : 512;
-  static_assert(TM_O + 2 * PVN <= TMEM_COLS, "tensor memory budget");
+  static constexpr uint32_t TM_P = 0;      // NPB P buffers of 32 columns (128 x 64 16-bit)
+  static constexpr uint32_t TM_O = (32 * NPB + 63) / 64 * 64;   // NOB O accumulators, PVN columns each
+  static constexpr uint32_t TMEM_COLS = TM_O + NOB * PVN <= 256 ? 256 : 512;
+  static_assert(TM_O + NOB * PVN <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -93,11 +116,11 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
   uint64_t* a_empty = a_full + C::STAGES;
   uint64_t* v_full = a_empty + C::STAGES;
   uint64_t* v_empty = v_full + C::STAGES;
-  uint64_t* p_full = v_empty + C::STAGES;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* o_full = p_empty + 2;    // [2] per O accumulator
-  uint64_t* o_empty = o_full + 2;    // [2] the accumulator's epilogue has read it
-  uint64_t* drain_bar = o_empty + 2;
+  uint64_t* p_full = v_empty + C::STAGES;   // [NPB] per P buffer
+  uint64_t* p_empty = p_full + C::NPB;
+  uint64_t* o_full = p_empty + C::NPB;      // [NOB] per O accumulator
+  uint64_t* o_empty = o_full + C::NOB;      // [NOB] the accumulator's epilogue has read it
+  uint64_t* drain_bar = o_empty + C::NOB;
   uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile uint32_t* abort_flag = misc + 1;
 
@@ -111,11 +134,11 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NPB; ++i) {
       mbar_init(&p_full[i], 4);
       mbar_init(&p_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NOB; ++i) {
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], 4);
     }
@@ -183,16 +206,16 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
       uint32_t c = 0, pc = 0, ui = 0;
       bool live = true;
       for (int u = u_first; u < p.units && live; u += u_step, ++ui) {
-        const uint32_t ob = ui & 1;
-        // the epilogue of tile ui - 2 must have read this accumulator
-        if (ui >= 2 && !mbar_wait_warp(&o_empty[ob], ((ui >> 1) - 1) & 1, kSiteOFull, abort_flag)) {
+        const uint32_t ob = ui % C::NOB;
+        // the epilogue of tile ui - NOB must have read this accumulator
+        if (ui >= C::NOB && !mbar_wait_warp(&o_empty[ob], (ui / C::NOB - 1) & 1, kSiteOFull, abort_flag)) {
           live = false;
           break;
         }
         const uint32_t o_tm = tmem + C::TM_O + ob * C::PVN;
         for (int kb = kb0; kb < kb1; ++kb, ++c, ++pc) {
           const uint32_t st = c % C::STAGES, n = c / C::STAGES;
-          const uint32_t pb = pc & 1, np = pc >> 1;
+          const uint32_t pb = pc % C::NPB, np = pc / C::NPB;
           if (!mbar_wait_warp(&v_full[st], n & 1, kSiteVFull, abort_flag)) { live = false; break; }
           if (!mbar_wait_warp(&p_full[pb], np & 1, kSitePFull, abort_flag)) { live = false; break; }
           tc_fence_after();
@@ -218,7 +241,7 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                // row of the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t g = static_cast<uint32_t>(warp - 2) >> 2;   // row group: key blocks c with c % 2 == g
+    const uint32_t g = static_cast<uint32_t>(warp - 2) >> 2;   // row group: key blocks c with c % RG == g
     uint32_t c = 0, pc = 0, ui = 0;
     bool live = true;
     for (int u = u_first; u < p.units && live; u += u_step, ++ui) {
@@ -232,7 +255,7 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
       }
       const float nl = -Lr * L2E;
       for (int kb = kb0; kb < kb1; ++kb, ++c, ++pc) {
-        if ((c & 1) != g) continue;   // the other group's block (P buffer c & 1 is this group's)
+        if (c % C::RG != g) continue;   // another group's block
         const uint32_t st = c % C::STAGES, n = c / C::STAGES;
         live = __all_sync(0xffffffffu, mbar_wait(&a_full[st], n & 1, kSiteAFull, abort_flag));
         if (!live) break;
@@ -284,7 +307,7 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_empty[st]);
-        const uint32_t pb = pc & 1, np = pc >> 1;
+        const uint32_t pb = pc % C::NPB, np = pc / C::NPB;
         live = __all_sync(0xffffffffu, mbar_wait(&p_empty[pb], (np & 1) ^ 1, kSitePEmpty, abort_flag));
         if (!live) break;
         tc_fence_after();
@@ -296,11 +319,11 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[pb]);
       }
       if (!live) break;
-      // ---- epilogue: O_i / S_i, by group ui & 1 ----
-      if ((ui & 1) != g) continue;
-      const uint32_t ob = ui & 1;
+      // ---- epilogue: O_i / S_i, by group ui % RG ----
+      if (ui % C::RG != g) continue;
+      const uint32_t ob = ui % C::NOB;
       const uint32_t o_tm = tmem + C::TM_O + ob * C::PVN + lane_off;
-      live = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (ui >> 1) & 1, kSiteOFull, abort_flag));
+      live = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (ui / C::NOB) & 1, kSiteOFull, abort_flag));
       if (!live) break;
       tc_fence_after();
       if (p.ksplit > 1) {
@@ -325,7 +348,7 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
       const int row_w = row - lane;   // the warp's first row
       uint8_t* owarp = reinterpret_cast<uint8_t*>(p.O) + (static_cast<int64_t>(bh) * p.N + row_w) * D * 2;
       // each row warp has a slice of its own: with one key block per tile the
-      // two groups finish alternate tiles at the same time
+      // groups finish consecutive tiles at the same time
       uint8_t* slice = smem + C::OFF_STG + (warp - 2) * RowStage<C::OCW>::BYTES;
 #pragma unroll
       for (int pass = 0; pass < D / C::OCW; ++pass) {
@@ -335,7 +358,7 @@ __global__ void __launch_bounds__(AVCfg<D, AF16>::NTHREADS, 1)
         tmem_wait_ld();
         reg_fence<C::OCW>(o);
         if (pass == D / C::OCW - 1) {
-          // the accumulator is read: the tile after next may overwrite it
+          // the accumulator is read: tile ui + NOB may overwrite it
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&o_empty[ob]);
