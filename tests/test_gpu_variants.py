@@ -102,6 +102,32 @@ def test_f16_stored_a(B, H, N, M, d):
     print(f"fp16 A {B, H, N, M, d}: max_abs {ea:.3e} rel_frob {er:.3e}")
 
 
+@pytest.mark.parametrize("d", [40, 80, 160])
+@pytest.mark.parametrize("variant", ["partial", "f16a"])
+def test_many_row_tiles_per_cta(d, variant):
+    """480 row tiles (3-4 per CTA of a persistent grid) of 5 key blocks each:
+    the second kernel's row groups take the blocks in turn and its O
+    accumulators rotate over the tiles of a CTA, every group and accumulator
+    in use with an odd number of blocks per tile."""
+    B, H, N, M = 1, 120, 512, 320
+    q, k, v, scale = _inputs(B, H, N, M, d, seed=17)
+    rows = np.unique(np.concatenate([np.arange(0, N, 37), np.arange(127, N, 128)]))
+    heads = np.arange(0, H, 7)
+    ref = oracle.attention(q[:, heads][:, :, rows], k[:, heads], v[:, heads], scale)
+    tq, tk, tv = (torch.from_numpy(x).to(DEV) for x in (q, k, v))
+    if variant == "partial":
+        a, ls = sd.qk_stats(tq, tk, scale)
+        o = sd.softmax_av(a, ls, tv, scale)
+    else:
+        a16, ls = sd.qk_stats_f16a(tq, tk, scale)
+        o = sd.softmax_av_f16a(a16, ls, tv, scale)
+    torch.cuda.synchronize()
+    got = o[:, torch.from_numpy(heads).to(DEV)][:, :, torch.from_numpy(rows).to(DEV)].float().cpu().numpy()
+    ea, er = gate(got, ref["O"], f"{variant} d={d}")
+    print(f"{variant} {B, H, N, M, d}: max_abs {ea:.3e} rel_frob {er:.3e}")
+    assert sd.device_error()[0] == "SDATTN_OK"
+
+
 def test_variants_on_64x64_self_sampled():
     """Full-size 64x64-latent self-attention, every tile sampled."""
     shape = synth.WORKLOADS["self64"]
