@@ -50,3 +50,19 @@ def test_both_arms_print_the_same_config():
     assert cfg["flops_per_step"] == bench.STEP_FLOPS and cfg["calls_per_step"] == 32
     assert bench.SET_BYTES > 126e6          # each input set is larger than the L2
     assert bench.job_config(1) == cfg
+
+
+def test_upload_groups_cover_the_calls_in_order():
+    """The end-to-end leg's upload runs: consecutive, disjoint, covering every
+    call once, at most the requested number, of about equal bytes."""
+    sizes = [2 * c.B * c.H * (c.N + 2 * c.M) * c.d for c in synth.unet_step_set()]
+    for groups in (1, 2, 4, 7, 32, 40):
+        runs = bench.upload_groups(sizes, groups)
+        assert runs[0][0] == 0 and runs[-1][1] == len(sizes)
+        assert all(a < b for a, b in runs)
+        assert all(runs[i][1] == runs[i + 1][0] for i in range(len(runs) - 1))
+        assert len(runs) <= groups
+    runs = bench.upload_groups(sizes, 4)
+    per = [sum(sizes[a:b]) for a, b in runs]
+    assert len(runs) == 4 and max(per) <= 1.25 * sum(sizes) / 4
+    assert bench.upload_groups([10], 4) == [(0, 1)]
