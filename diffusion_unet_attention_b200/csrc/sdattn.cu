@@ -169,7 +169,10 @@ CUtensorMapDataType elem_type(const sdattn_desc* d) {
 }
 
 // Column splits of the statistics reduction: the smallest power of two that
-// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit.
+// fills the SMs evenly (at least 90% of the last wave), at most kMaxSplit;
+// a split that takes the grid past one wave must also shorten the busiest
+// CTA's chain (at 32x32, 128 row tiles of 8 blocks: two splits leave 8
+// blocks on the busiest CTA and add two hand-offs).
 // A split keeps at least kMinBlocksPerSplit column blocks (each split pays a
 // partial write and an arrival, which a one-block split cannot hide on a busy
 // GPU), except while the doubled grid still fills at most half of the SMs:
@@ -188,10 +191,19 @@ QKPlan plan_qk(const sdattn_desc* d, int nsm) {
     const int64_t waves = (u + nsm - 1) / nsm;
     return static_cast<double>(u) / static_cast<double>(waves * nsm);
   };
+  // A CTA's chain, in block times of one epilogue group: its units in turn,
+  // each its blocks shared by the epilogue groups plus, when split, the
+  // hand-off of the partial statistics (about one block time, measured).
+  const int epi = (d->d + 63) / 64 == 3 ? 1 : 2;   // epilogue groups at this head width
+  auto chain = [&](int ns) {
+    const int cbs = (pl.nb + ns - 1) / ns;
+    const int64_t units = base * ((pl.nb + cbs - 1) / cbs);
+    return (units + nsm - 1) / nsm * ((cbs + epi - 1) / epi + (ns > 1 ? 1 : 0));
+  };
   int ns = 1;
   const int cap = pl.nb < kMaxSplit ? pl.nb : kMaxSplit;
   while (ns * 2 <= cap && (pl.nb / (ns * 2) >= kMinBlocksPerSplit || base * ns * 2 <= nsm / 2) &&
-         eff(base * ns) < 0.9)
+         eff(base * ns) < 0.9 && (base * ns * 2 <= nsm || chain(ns * 2) < chain(ns)))
     ns *= 2;
   pl.cbs = (pl.nb + ns - 1) / ns;
   pl.nsplit = (pl.nb + pl.cbs - 1) / pl.cbs;

@@ -51,9 +51,9 @@ def _run(lib, fn, desc, tq, tk, lda, ws=None):
 # Column splits with 148 SMs in brackets (the plan depends on the SM count).
 @pytest.mark.parametrize("B,H,N,M,d", [
     (1, 4, 128, 8192, 40),      # [16 splits] four row tiles of partials and counters
-    (2, 8, 512, 4096, 40),      # [8 splits]
+    (2, 8, 512, 4096, 40),      # [2 splits]
     (2, 8, 4096, 4096, 40),     # [2 splits] 64x64-latent self-attention
-    (2, 8, 1024, 1024, 80),     # [2 splits] 32x32-latent self-attention
+    (2, 8, 1024, 1024, 80),     # [1 split] 32x32-latent self-attention: one wave unsplit
     (2, 8, 300, 77, 160),       # [1 split] no scratch in use
 ])
 def test_matches_workspace_entry_point_twice(B, H, N, M, d):
@@ -74,15 +74,16 @@ def test_matches_workspace_entry_point_twice(B, H, N, M, d):
 
 
 def test_rejects_shapes_beyond_its_scratch():
-    """149 row tiles of 8192-key rows: with 148 SMs the plan splits each row 16
-    ways, whose partials (about 2.4 MB) exceed the 2 MiB array.  The split plan
-    follows the SM count, so the case is only known to exceed it on 148 SMs.
-    The buffers are real and full-size, so a call that were accepted would
-    still stay inside them."""
+    """1060 row tiles of 16384-key rows: with 148 SMs the plan splits each row
+    in two (the split shortens the busiest CTA's chain from 512 to 495 block
+    times), and the partials (1060 x 128 x 2 float2, 2.17 MB) exceed the 2 MiB
+    array.  The split plan follows the SM count, so the case is only known to
+    exceed it on 148 SMs.  The buffers are real and full-size, so a call that
+    were accepted would still stay inside them."""
     if torch.cuda.get_device_properties(DEV).multi_processor_count != 148:
         pytest.skip("the split plan of this shape is worked out for 148 SMs")
     lib = _lib.load()
-    B, H, N, M, d = 1, 149, 128, 8192, 40
+    B, H, N, M, d = 1, 1060, 128, 16384, 40
     desc = _lib.Desc(B, H, N, M, d, _lib.SDATTN_F16, 0.15811388)
     q = torch.zeros((B, H, N, d), dtype=torch.float16, device=DEV)
     k = torch.zeros((B, H, M, d), dtype=torch.float16, device=DEV)
