@@ -766,6 +766,12 @@ sdattn_status dispatch_flash(const sdattn_desc* d, const void* Q, const void* K,
   const bool two = pairs >= nsm;   // enough work for two query tiles per CTA
   switch (d->d) {
     case 40:
+      // keys that fit one 96-key tile (cross-attention, 77 text tokens): a
+      // narrower score tile, so the exponentials, row max and products cover
+      // 96 columns instead of 128
+      if (d->M <= 96)
+        return two ? launch_flash<40, 2, 96, BF16>(d, Q, K, V, O, LS, ws, s)
+                   : launch_flash<40, 1, 96, BF16>(d, Q, K, V, O, LS, ws, s);
       return two ? launch_flash<40, 2, 128, BF16>(d, Q, K, V, O, LS, ws, s)
                  : launch_flash<40, 1, 128, BF16>(d, Q, K, V, O, LS, ws, s);
     case 80:
