@@ -62,7 +62,7 @@ def parse_args():
                     help="time the step set only (no per-form, per-kernel or end-to-end extras)")
     ap.add_argument("--case", default=None,
                     help="FORM:WORKLOAD, e.g. flash:self64 -- run one form (flash, qk_stats, softmax_av, "
-                         "qk_stats_f16a, softmax_av_f16a, partial, f16a, or all three kernels) on one workload; or conv3x3:CxH, e.g. conv3x3:320x64 -- one "
+                         "qk_stats_f16a, softmax_av_f16a, partial, f16a, three_pass, or all three kernels) on one workload; or conv3x3:CxH, e.g. conv3x3:320x64 -- one "
                          "Winograd 3x3 convolution (batch 2, C = K) (for profilers)")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
@@ -927,6 +927,8 @@ def run_case(args):
         elif form == "f16a":    # the fp16-A variant's two kernels
             sd.qk_stats_f16a(tq, tk, scale, out_a=a16, out_ls=ls, ws=scratch.ws)
             sd.softmax_av_f16a(a16, ls, tv, scale, out=o)
+        elif form == "three_pass":    # A alone, the stand-alone reduction, softmax_av
+            scratch.run(call, tq, tk, tv, o, "three_pass")
         else:
             scratch.run(call, tq, tk, tv, o, "partial")
 
