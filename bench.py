@@ -370,6 +370,7 @@ def run_gpu(args, rank, world, local_rank):
         extra["per_call"] = per_call_table(torch, sd, stream, sets, scratch)
         extra["unet_ops"] = unet_ops_table(torch, sd, stream)
         extra["conv3x3_winograd"] = conv3x3_table(torch, sd, stream)
+        extra["dtype_forms"] = dtype_forms_table(torch, sd, stream)
     if not args.no_side:
         # every rank feeds its own replica from host memory; the job's step is its slowest rank's
         barrier()
@@ -682,6 +683,70 @@ def conv3x3_table(torch, sd, stream, reps=20):
         del xs, ys, U, ws
     return {"note": f"graph of {reps} calls over buffers totalling > 256 MB; fp16, fp32 accumulation; filter "
                     "transformed once outside the timed region", "rows": rows}
+
+
+def dtype_forms_table(torch, sd, stream, reps=20):
+    """The forms for other input types: bf16 inputs with fp32 O (P carried in
+    two 16-bit parts, two P V products), plain bf16 flash beside it, and fp32
+    inputs through tf32 products, on the 64x64 self-attention and the tiny
+    fp32 configuration.  Each is a graph of `reps` launches cycling over input
+    sets that total more than 256 MB.  FLOPs are the algorithmic 4 B H N M d;
+    the tf32 peak is the measured bf16 dense peak times the nominal
+    tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s)."""
+    peaks, _ = measured_peaks()
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rows = []
+
+    def timed(issue, nbuf):
+        for r in range(3):
+            issue(r % nbuf)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    issue(r % nbuf)
+            g.replay()
+            ts = []
+            for _ in range(3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                stream.synchronize()
+                ts.append(a.elapsed_time(b) / reps)
+        del g
+        return statistics.median(ts)
+
+    cases = [("flash_f32o", "self64", torch.bfloat16), ("flash", "self64", torch.bfloat16),
+             ("flash_tf32", "self64", torch.float32), ("flash_tf32", "tiny", torch.float32)]
+    for form, wl, dtype in cases:
+        c = synth.WORKLOADS[wl]
+        per_set = c.B * c.H * (c.N + 2 * c.M) * c.d * (4 if dtype == torch.float32 else 2) + c.B * c.H * c.N * c.d * 4
+        nbuf = max(2, math.ceil(256e6 / per_set))
+        gen = torch.Generator(device=dev).manual_seed(c.d + c.N)
+        sets = []
+        for _ in range(nbuf):
+            q = torch.randn(c.B, c.H, c.N, c.d, device=dev, generator=gen).to(dtype)
+            k = torch.randn(c.B, c.H, c.M, c.d, device=dev, generator=gen).to(dtype)
+            v = torch.randn(c.B, c.H, c.M, c.d, device=dev, generator=gen).to(dtype)
+            o = torch.empty(c.B, c.H, c.N, c.d, device=dev,
+                            dtype=dtype if form == "flash" else torch.float32)
+            sets.append((q, k, v, o))
+        scale = 1.0 / math.sqrt(c.d)
+        fn = getattr(sd, form)
+        with torch.cuda.stream(stream):
+            ms = timed(lambda i: fn(sets[i][0], sets[i][1], sets[i][2], scale, out=sets[i][3]), nbuf)
+        flops = 4 * c.B * c.H * c.N * c.M * c.d
+        peak = bf16_peak * (1.1 / 2.25 if dtype == torch.float32 else 1.0)
+        tflops = flops / (ms * 1e-3) / 1e12
+        rows.append({"form": form, "workload": wl, "inputs": str(dtype).replace("torch.", ""),
+                     "shape": [c.B, c.H, c.N, c.M, c.d], "us": round(ms * 1e3, 2), "tflops": round(tflops, 1),
+                     "peak_tflops": round(peak, 1), "frac_peak": round(tflops / peak, 4)})
+        del sets
+    return {"note": f"graph of {reps} launches over inputs totalling > 256 MB; tf32 peak = measured bf16 x 1.1/2.25",
+            "rows": rows}
 
 
 def upload_groups(sizes, groups):

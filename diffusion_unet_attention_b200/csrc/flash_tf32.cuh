@@ -25,7 +25,7 @@
 // row d of V^T holds ones, so column d of O accumulates the row sum; rows
 // d .. PVN - 1 are written once.
 // One 128-row query tile per CTA, persistent over the (b*H + h, row tile)
-// units; roles: warp 0 TMA, warp 1 MMA, warps 2..3 operand preparation (Q
+// units; roles: warp 0 TMA, warp 1 MMA, warps 2, 3, 8, 9 operand preparation (Q
 // and K rounded to tf32 in place, V transposed and rounded), warps 4..7
 // softmax (one row per thread), with S, P (fp32, BN columns) and O in tensor
 // memory.
@@ -82,9 +82,13 @@ struct FlashTF32Cfg {
   static constexpr int K_BYTES = DSL * KV_SLAB;
   static constexpr int V_BYTES = DSL * KV_SLAB;
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int STAGES = 2;
   static constexpr int VT_SLAB = PVN * 128;                // 32 keys of PVN rows
   static constexpr int VT_STAGE = (BN / 32) * VT_SLAB;
+  // as many K / V / V^T stages as fit (at most 4): loads run that many key
+  // tiles ahead of the preparation, products and softmax
+  static constexpr int STAGES_FIT = (232448 - Q_BYTES - 1024 - 16 - 8 * (8 + 5 * 4)) / (STAGE + VT_STAGE);
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
+  static_assert(STAGES >= 2, "key / value ring too shallow");
   static constexpr uint32_t TM_S = 0, TM_P = BN, TM_O = 2 * BN;
   static constexpr uint32_t TMEM_COLS = TM_O + PVN <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
@@ -93,7 +97,10 @@ struct FlashTF32Cfg {
   static constexpr int OFF_BAR = OFF_VT + STAGES * VT_STAGE;
   static constexpr int NBAR = 3 + 5 * STAGES + 5;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr int NTHREADS = 256;
+  // preparation warps 2, 3, 8, 9: measured at 64x64, 2 -> 4 warps took the
+  // call from 440 to 336 us; 6 or 8 gave nothing more
+  static constexpr int NPREP = 4;
+  static constexpr int NTHREADS = 256 + 32 * (NPREP - 2);
   static_assert(D % 8 == 0 && BN % 32 == 0, "whole MMA K steps, whole V^T slabs");
   static_assert(TM_O + PVN <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -143,13 +150,13 @@ __global__ void __launch_bounds__(FlashTF32Cfg<D>::NTHREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    mbar_init(q_ready, 2);
+    mbar_init(q_ready, C::NPREP);
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
-      mbar_init(&vt_full[i], 2);
-      mbar_init(&k_ready[i], 2);
+      mbar_init(&vt_full[i], C::NPREP);
+      mbar_init(&k_ready[i], C::NPREP);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
@@ -261,15 +268,26 @@ __global__ void __launch_bounds__(FlashTF32Cfg<D>::NTHREADS, 1)
     volatile uint32_t never = 0;
     mma_commit(drain_bar);
     mbar_wait_warp(drain_bar, 0, kSitePvDone, &never);
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 2 || warp == 3 || warp >= 8) {
     // ------------------------- operand preparation --------------------------
     // Q and K rounded to tf32 in place; V [key r][column c] (as loaded:
     // 32-column slabs, 128-byte swizzled) -> V^T [row c][key r] (32-key slabs,
     // 128-byte swizzled), rows 0 .. D - 1, rounded to tf32.
-    const int tid = threadIdx.x - 64;
+    const int tid = warp >= 8 ? static_cast<int>(threadIdx.x) - 192 : static_cast<int>(threadIdx.x) - 64;
+    constexpr int kPrepThreads = 32 * C::NPREP;
+    // 16 bytes per access (the swizzle moves whole 16-byte chunks, so the
+    // rounding does not care where a word sits)
     auto round_in_place = [&](uint8_t* base, int words) {
-      uint32_t* w = reinterpret_cast<uint32_t*>(base);
-      for (int i = tid; i < words; i += 64) w[i] = round_tf32(__uint_as_float(w[i]));
+      uint4* w = reinterpret_cast<uint4*>(base);
+#pragma unroll 4
+      for (int i = tid; i < words / 4; i += kPrepThreads) {
+        uint4 x = w[i];
+        x.x = round_tf32(__uint_as_float(x.x));
+        x.y = round_tf32(__uint_as_float(x.y));
+        x.z = round_tf32(__uint_as_float(x.z));
+        x.w = round_tf32(__uint_as_float(x.w));
+        w[i] = x;
+      }
     };
     auto publish = [&](uint64_t* bar) {
       fence_proxy_async_smem();   // generic-proxy writes before the tensor core reads them
@@ -294,17 +312,28 @@ __global__ void __launch_bounds__(FlashTF32Cfg<D>::NTHREADS, 1)
         if (!live) break;
         const uint8_t* sV = sK + C::K_BYTES;
         uint8_t* vt = sVT + st * C::VT_STAGE;
-        for (int idx = tid; idx < D * BN; idx += 64) {
-          const int c = idx / BN, r = idx - c * BN;
-          const float val = *reinterpret_cast<const float*>(
-              sV + (c >> 5) * C::KV_SLAB + r * 128 + ((((c & 31) >> 2) ^ (r & 7)) << 4) + (c & 3) * 4);
-          *reinterpret_cast<uint32_t*>(vt + (r >> 5) * C::VT_SLAB + c * 128 + ((((r & 31) >> 2) ^ (c & 7)) << 4) +
-                                       (r & 3) * 4) = round_tf32(val);
+        // one item = key r, columns c4 .. c4 + 3: a 16-byte chunk of V's row
+        // (consecutive lanes take consecutive keys: eight lanes cover the
+        // eight chunk positions of the swizzle, no bank conflicts), four
+        // rounded words into four rows of V^T
+#pragma unroll 2
+        for (int idx = tid; idx < (D / 4) * BN; idx += kPrepThreads) {
+          const int c4 = (idx / BN) * 4, r = idx - (idx / BN) * BN;
+          const uint4 x = *reinterpret_cast<const uint4*>(sV + (c4 >> 5) * C::KV_SLAB + r * 128 +
+                                                          ((((c4 & 31) >> 2) ^ (r & 7)) << 4));
+          const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
+          uint8_t* vrow = vt + (r >> 5) * C::VT_SLAB + (r & 3) * 4;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = c4 + i;
+            *reinterpret_cast<uint32_t*>(vrow + c * 128 + ((((r & 31) >> 2) ^ (c & 7)) << 4)) =
+                round_tf32(__uint_as_float(xv[i]));
+          }
         }
         publish(&vt_full[st]);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ---------------------------- softmax, one row per thread -----------------------------
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
