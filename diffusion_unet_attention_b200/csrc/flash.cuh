@@ -32,7 +32,9 @@
 // every stage (written once; the V tile loads never cover it), so column D of
 // O accumulates sum_j p_j from the same 16-bit P that multiplies V.
 //
-// Precise variant (template flag PREC, one query tile per CTA): P is carried
+// Precise variant (template flag PREC; two query tiles per CTA only with
+// 96-key tiles, which leave room in tensor memory for both tiles' S, P, P's
+// residual and O): P is carried
 // as a 16-bit high part plus the 16-bit rounding of its residual, P V runs as
 // two MMAs into the same accumulator, and O is written in fp32.  Both parts
 // have the input's type, so with bf16 inputs (8-bit mantissas) the weights
@@ -184,7 +186,7 @@ struct FlashCfg {
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 128, "key tile");
   static_assert(TAIL % 8 == 0 && TAIL < 64, "room for the ones column in V's last slab");
   static_assert((PREC ? 2 * D : D) % OCW == 0, "whole store passes");
-  static_assert(!PREC || NQ == 1, "the precise variant keeps one query tile per CTA");
+  // the precise variant never cuts a unit (it runs without the split schedule)
   static_assert(NQ > 1 || 128 * (D + 4) * 4 <= STAGES * STAGE, "cluster partial rows fit in the key/value stages");
 };
 

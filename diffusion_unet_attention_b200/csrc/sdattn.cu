@@ -745,12 +745,19 @@ sdattn_status launch_flash_tf32(const sdattn_desc* d, const void* Q, const void*
   return launch(kern, grid, C::NTHREADS, C::SMEM, stream, mq, mk, mv, p) ? SDATTN_OK : SDATTN_ERR_CUDA;
 }
 
-// The precise variant: one query tile per CTA, every block of rows whole.
+// The precise variant: every block of rows whole; at d = 40 with enough work,
+// two query tiles per CTA over 96-key tiles (tensor memory holds S, P, P's
+// residual and O of both), else one query tile over 128-key tiles.
 template <bool BF16>
 sdattn_status dispatch_flash_f32o(const sdattn_desc* d, const void* Q, const void* K, const void* V, float* O,
                                   float* LS, cudaStream_t s) {
+  const int dev = current_device();
+  const int nsm = sm_count(dev < 0 ? 0 : dev);
+  const int64_t pairs = static_cast<int64_t>(d->B) * d->H * ((d->N + 255) / 256);
   switch (d->d) {
-    case 40: return launch_flash<40, 1, 128, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
+    case 40:
+      if (pairs >= nsm) return launch_flash<40, 2, 96, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
+      return launch_flash<40, 1, 128, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
     case 80: return launch_flash<80, 1, 128, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
     case 160: return launch_flash<160, 1, 64, BF16, 3, true>(d, Q, K, V, O, LS, nullptr, s);
   }
